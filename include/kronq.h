@@ -1,0 +1,265 @@
+/*
+ * kronq.h — C ABI of libkronq.so, the per-sublayer quantization engine of
+ * KronQ (Kronecker-factored-Hessian post-training quantization) for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources (web pages about arXiv 2607.07964, "KronQ: LLM Quantization via
+ * Kronecker-Factored Hessian"), cited below by these short names:
+ *   [gptget-en]  gptget.net, "KronQ: LLM Quantization via Kronecker-Factored
+ *                Hessian" (English summary): Methodology, Technical
+ *                Contribution, Novelty, Abstract.
+ *   [gptget-zh]  gptget.net, same title, Chinese summary: 方法论, 技术贡献.
+ *   [aimodeling] aimodeling.com news, "KronQ：Kronecker Hessian 拆掉 GPTQ 的
+ *                2-bit 墙" (English title "KronQ: Kronecker Hessians break
+ *                GPTQ's 2-bit wall").
+ *   [wmrh]       wmrh.cn long-form article on KronQ, sections 一 … 九 and the
+ *                closing Q&A (Q1–Q3).
+ *
+ * The engine, per linear sublayer W (d_out x d_in, y = W x):
+ *   1. covariances  H_X = X^T X / n,  H_G = G^T G / n      [wmrh §二; aimodeling]
+ *   2. sensitivity  tr(H_G) * tr(H_X)                      [wmrh §三, §六; aimodeling]
+ *   3. BiIP: diagonal rescale from diag(H_X), diag(H_G), then a seeded
+ *      orthogonal rotation on both sides of W, H_X and H_G rotated to match
+ *                                                          [wmrh §三, §八, Q2; aimodeling]
+ *   4. damped Cholesky factor U of H_X'^{-1} (H_G is not needed after 3,
+ *      because it cancels from the per-column update)      [wmrh §四, §七]
+ *   5. GPTQ-style column-wise OBS quantize-and-compensate with asymmetric
+ *      min-max group scales at 2/3/4 bits                  [gptget-en Methodology; wmrh §四, §五]
+ *   plus a greedy mixed-precision bit allocator driven by step 2 [wmrh §六].
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions (all entry points except kronq_allocate_bits and
+ * kronq_status_string):
+ *   - Every pointer is a DEVICE pointer owned by the caller. The library never
+ *     allocates device memory; scratch space is passed as (ws, ws_bytes), sized
+ *     by kronq_workspace_bytes(). ws must be 256-byte aligned.
+ *   - Every matrix is row-major and dense. d_out x d_in means d_out rows.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Inputs must stay alive until the stream reaches the
+ *     call.
+ *   - The return value reports argument, shape and launch errors only.
+ *     Numerical outcomes go to the device int32 word *info_dev, which the
+ *     call first sets to 0 (stream-ordered). After synchronising, the caller
+ *     reads it: 0 = ok; (KRONQ_ERR_NOT_PD | (col << 8)) when the damped
+ *     Cholesky meets a pivot <= 0 or non-finite at column `col`;
+ *     KRONQ_ERR_NONFINITE when an input holds a NaN/Inf the call checks for.
+ *   - There is no CPU fallback: without a usable CUDA device every call
+ *     returns KRONQ_ERR_CUDA.
+ * ---------------------------------------------------------------------------
+ * Rotation and random-number specification (BiIP, step 3).
+ *
+ * [wmrh §三, §七, Q2] realise the two-sided incoherence rotation as a
+ * bidirectional Hadamard transform; [wmrh §八] puts a diagonal scaling from
+ * diag(H_X), diag(H_G) before it. The pages give neither the scaling exponent
+ * nor the construction for sizes that are not powers of two; the library
+ * fixes them as follows (both the GPU path and the test oracle implement this
+ * text independently).
+ *
+ *   splitmix64 (Steele, Lea & Flood 2014; reference C by S. Vigna): for a
+ *   64-bit state s, sm64(s) = mix(s + 0x9E3779B97F4A7C15) with
+ *     mix(z): z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9;
+ *             z = (z ^ (z >> 27)) * 0x94D049BB133111EB;
+ *             return z ^ (z >> 31);            (all arithmetic mod 2^64)
+ *   so sm64(0) = 0xE220A8397B1DCDAF is the generator's first output for seed 0.
+ *
+ *   Per side (side = 0 for the input dimension d_in, 1 for the output
+ *   dimension d_out): key = sm64(sm64(seed) + side).
+ *   Size d = had * m with had a power of two and 1 <= m <= 256.
+ *   Index i in [0, d) splits as i = a*m + b, a in [0, had), b in [0, m).
+ *     sign_i = +1 if bit 63 of sm64(key + i) is 0, else -1.
+ *     Q_m: let kq = key ^ 0xA5A5A5A5A5A5A5A5. For t = r*m + c (r, c in [0,m)):
+ *       u1 = ((sm64(kq + 2t) >> 11) + 1) * 2^-53          in (0, 1]
+ *       u2 =  (sm64(kq + 2t + 1) >> 11) * 2^-53           in [0, 1)
+ *       G[r][c] = sqrt(-2 ln u1) * cos(2 pi u2)            (Box–Muller)
+ *     Q_m is the orthogonal factor of the QR factorisation G = Q_m R with
+ *     every R[j][j] > 0 (unique; computed in fp64). For m = 1, Q_1 = [1].
+ *   Hhat = Sylvester Hadamard of order had (Hhat[a][a'] = (-1)^popcount(a&a'))
+ *          divided by sqrt(had).
+ *   The side's rotation is U = (Hhat kron Q_m) * diag(sign):
+ *     (U v)[a*m + b] = sum_{a',b'} Hhat[a][a'] * Q_m[b][b'] * sign[a'*m+b'] * v[a'*m+b'].
+ *   Diagonal scale: s_i = max(h_ii, 1e-8 * mean(diag h))^scale_exp, with h the
+ *   side's covariance (H_X for the input side, H_G for the output side).
+ *
+ *   BiIP then produces
+ *     W'   = U_G * S_G * W * S_X * U_X^T
+ *     H_X' = U_X * S_X^-1 * H_X * S_X^-1 * U_X^T
+ *     H_G' = U_G * S_G^-1 * H_G * S_G^-1 * U_G^T
+ *   so that tr(H_G' dW' H_X' dW'^T) = tr(H_G dW H_X dW^T) for every dW.
+ * ---------------------------------------------------------------------------
+ * Quantizer (step 5), per row and per group of `group` consecutive input
+ * columns, evaluated on the row's current (compensated) weights at the
+ * group's first column [wmrh §五: W2/W3/W4, g128]:
+ *   xmin = min(0, min w), xmax = max(0, max w)
+ *   if xmax == xmin: scale = 1, zero = 0
+ *   else:            scale = (xmax - xmin) / (2^bits - 1), zero = rint(-xmin / scale)
+ *   q = clamp(rint(w / scale) + zero, 0, 2^bits - 1),  w_hat = scale * (q - zero)
+ *   (rint = round half to even). Then, with U the upper Cholesky factor of
+ *   (H_X' + lambda I)^-1:  err = (w_j - w_hat_j) / U[j][j];
+ *   w_k -= err * U[j][k] for every k > j of the row.  H_G does not appear
+ *   [wmrh §四].
+ * Packed codes: per row a little-endian bitstream of d_in codes, code of
+ *   column c in bits [c*bits, c*bits + bits) of the row; the row occupies
+ *   bits*d_in/32 uint32 words (d_in % 32 == 0 is required).
+ * ---------------------------------------------------------------------------
+ */
+#ifndef KRONQ_H
+#define KRONQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kronq_stream_t; /* ABI-identical to cudaStream_t */
+
+typedef enum {
+  KRONQ_OK = 0,
+  KRONQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad dtype     */
+  KRONQ_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes     */
+  KRONQ_ERR_NOT_PD = 3,      /* info word only: pivot <= 0 (col in b8..31) */
+  KRONQ_ERR_NONFINITE = 4,   /* info word only: NaN/Inf met               */
+  KRONQ_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up         */
+  KRONQ_ERR_CUDA = 6         /* a CUDA launch or runtime call failed       */
+} kronq_status;
+
+typedef enum { KRONQ_F32 = 0, KRONQ_BF16 = 1 } kronq_dtype;
+
+/* Factorisation of one side's dimension d = had * m (see the spec above). */
+typedef struct {
+  int64_t had; /* power of two, >= 1 */
+  int64_t m;   /* 1 <= m <= 256      */
+} kronq_rot;
+
+/* flags for kronq_opts.flags */
+#define KRONQ_FLAG_NO_ROT_IN   0x1u /* skip U_X (input-side rotation)  */
+#define KRONQ_FLAG_NO_ROT_OUT  0x2u /* skip U_G (output-side rotation) */
+#define KRONQ_FLAG_NO_SCALE    0x4u /* S_X = S_G = I                   */
+
+typedef struct {
+  int32_t bits;      /* 2, 3 or 4                                          */
+  int32_t group;     /* 32, 64 or 128; divides d_in                        */
+  int32_t block;     /* OBS block width; must be 128                       */
+  float damp_rel;    /* lambda = damp_rel * mean(diag H_X')                */
+  float scale_exp;   /* exponent of the diagonal scale (0.25 by default)   */
+  uint64_t seed;     /* BiIP seed                                          */
+  kronq_rot rot_in;  /* d_in  = rot_in.had  * rot_in.m                     */
+  kronq_rot rot_out; /* d_out = rot_out.had * rot_out.m                    */
+  uint32_t flags;    /* KRONQ_FLAG_*                                       */
+} kronq_opts;
+
+/* Which call a workspace size is asked for. */
+typedef enum {
+  KRONQ_WS_BIIP = 0,
+  KRONQ_WS_CHOL = 1,
+  KRONQ_WS_QUANT = 2,
+  KRONQ_WS_LOSS = 3
+} kronq_ws_kind;
+
+/*
+ * Step 1 — calibration covariance [wmrh §二; aimodeling; gptget-en Methodology:
+ * H_G from one backward pass].
+ *   H = alpha * A^T A + beta * H
+ * A: n x d (row stride lda elements, lda >= d), dtype KRONQ_BF16 (tensor-core
+ * path, fp32 accumulation) or KRONQ_F32 (fp32 path). H: d x d fp32, both
+ * triangles written. For one pass over all rows use alpha = 1/n, beta = 0
+ * (H need not be initialised then). BF16 needs d % 128 == 0 and lda % 8 == 0
+ * and a 16-byte aligned A; otherwise KRONQ_ERR_UNSUPPORTED. n == 0 scales H by
+ * beta. Symmetric in its result; the two triangles are written from the same
+ * accumulator tile, so they are bitwise equal.
+ */
+kronq_status kronq_accum_cov(kronq_stream_t stream, const void *A,
+                             kronq_dtype dtype, int64_t n, int64_t d,
+                             int64_t lda, float alpha, float beta, float *H);
+
+/*
+ * Step 2 — sublayer sensitivity [wmrh §三, §六; aimodeling].
+ * out_dev[0] = tr(H_X), out_dev[1] = tr(H_G), out_dev[2] = their product,
+ * summed in fp64 from the fp32 diagonals. Call it on the covariances BEFORE
+ * kronq_biip (the rotation keeps traces, the diagonal rescale does not).
+ */
+kronq_status kronq_sensitivity(kronq_stream_t stream, const float *H_X,
+                               int64_t d_in, const float *H_G, int64_t d_out,
+                               double *out_dev);
+
+/*
+ * Step 3 — bidirectional incoherence processing [wmrh §三, §八, Q2;
+ * aimodeling; gptget-en Technical Contribution]. See the spec above.
+ * W: d_out x d_in (dtype wdtype, read only). W_rot: d_out x d_in fp32 output.
+ * H_X (d_in^2) and H_G (d_out^2): full symmetric fp32, rotated in place.
+ * s_x[d_in], s_g[d_out]: fp32 outputs, the diagonal scales used (all 1 with
+ * KRONQ_FLAG_NO_SCALE). ws: kronq_workspace_bytes(KRONQ_WS_BIIP, ...).
+ * Requires d_in % 32 == 0, had*m == d per side, had a power of two,
+ * 1 <= m <= 256, d <= 65536. info: NONFINITE when a diagonal is not finite.
+ */
+kronq_status kronq_biip(kronq_stream_t stream, const kronq_opts *opts,
+                        const void *W, kronq_dtype wdtype, int64_t d_out,
+                        int64_t d_in, float *W_rot, float *H_X, float *H_G,
+                        float *s_x, float *s_g, void *ws, size_t ws_bytes,
+                        int32_t *info_dev);
+
+/*
+ * Step 4 — damped inverse Cholesky factor [wmrh §四; GPTQ-style OBS needs
+ * the upper factor of the inverse Hessian].
+ * In: H (d x d fp32, full symmetric, e.g. H_X'). Out, in place: U upper
+ * triangular with U^T U = (H + lambda I)^-1, lambda = damp_rel * mean(diag H),
+ * strict lower triangle set to 0. Computed as H + lambda I = R R^T (R upper,
+ * reverse-order Cholesky) and U = R^-1, in fp32 with 3xTF32 tensor-core
+ * trailing updates. Requires d % 128 == 0. info: NOT_PD with the column.
+ */
+kronq_status kronq_chol_inv(kronq_stream_t stream, float *H, int64_t d,
+                            float damp_rel, void *ws, size_t ws_bytes,
+                            int32_t *info_dev);
+
+/*
+ * Step 5 — blocked column-wise OBS quantization [gptget-en Methodology;
+ * wmrh §四, §五]. See the quantizer spec above.
+ * W_rot: d_out x d_in fp32; in: the weights to quantize (W' after BiIP);
+ * out: the dequantized weights w_hat. U: d_in x d_in from kronq_chol_inv.
+ * codes: d_out x (bits*d_in/32) uint32. scales: d_out x (d_in/group) fp32.
+ * zeros: d_out x (d_in/group) uint8. opts: bits, group, block used.
+ * Requires d_in % 128 == 0.
+ */
+kronq_status kronq_quantize_sublayer(kronq_stream_t stream,
+                                     const kronq_opts *opts, float *W_rot,
+                                     const float *U, int64_t d_out,
+                                     int64_t d_in, uint32_t *codes,
+                                     float *scales, uint8_t *zeros, void *ws,
+                                     size_t ws_bytes, int32_t *info_dev);
+
+/*
+ * Measurement — the Kronecker-factored layer loss [aimodeling: H ≈ H_X ⊗ H_G;
+ * wmrh §二]: *loss_dev = tr(H_G dW H_X dW^T) with dW = W_ref - W_hat, summed in
+ * fp64 over fp32 products (3xTF32 tensor-core GEMMs). d_in, d_out % 128 == 0.
+ */
+kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
+                              const float *W_hat, const float *H_X,
+                              const float *H_G, int64_t d_out, int64_t d_in,
+                              double *loss_dev, void *ws, size_t ws_bytes);
+
+/* Workspace bytes needed by one call (opts may be NULL except for BIIP and
+ * QUANT). Returns 0 for unsupported arguments. */
+size_t kronq_workspace_bytes(kronq_ws_kind which, int64_t d_out, int64_t d_in,
+                             const kronq_opts *opts);
+
+/*
+ * Mixed-precision bit allocation [wmrh §六: upgrade the most sensitive
+ * sublayers first]. HOST pointers. All sublayers start at 2 bits; pass 1
+ * visits them in descending score (ties: lower index first) and upgrades
+ * 2 -> 3 when the parameter-weighted mean bit width stays <= avg_budget;
+ * pass 2 does the same for 3 -> 4. bits_out[i] in {2,3,4}.
+ * KRONQ_ERR_INVALID_ARG for n <= 0, null pointers, numel <= 0, non-finite
+ * scores or avg_budget < 2.
+ */
+kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,
+                                 int n, double avg_budget, int *bits_out);
+
+/* Static, human-readable name of a status code. */
+const char *kronq_status_string(kronq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRONQ_H */
