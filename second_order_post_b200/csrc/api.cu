@@ -1,0 +1,199 @@
+// The C ABI of libkronq.so (declared in include/kronq.h): argument validation
+// and dispatch to the kernels. No call allocates device memory.
+#include <math.h>
+
+#include <algorithm>
+#include <numeric>
+#include <vector>
+
+#include "kernels.cuh"
+
+using namespace kronq;
+
+namespace {
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+bool rot_ok(const kronq_rot &r, int64_t d) {
+  return is_pow2(r.had) && r.m >= 1 && r.m <= 256 && r.had * r.m == d;
+}
+
+bool aligned(const void *p, size_t a) {
+  return reinterpret_cast<uintptr_t>(p) % a == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kronq_status_string(kronq_status s) {
+  switch (s) {
+    case KRONQ_OK: return "ok";
+    case KRONQ_ERR_INVALID_ARG: return "invalid argument";
+    case KRONQ_ERR_UNSUPPORTED: return "unsupported shape or layout";
+    case KRONQ_ERR_NOT_PD: return "matrix not positive definite";
+    case KRONQ_ERR_NONFINITE: return "non-finite value";
+    case KRONQ_ERR_TIMEOUT: return "device wait timed out";
+    case KRONQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+kronq_status kronq_accum_cov(kronq_stream_t stream, const void *A,
+                             kronq_dtype dtype, int64_t n, int64_t d,
+                             int64_t lda, float alpha, float beta, float *H) {
+  if (!H || d <= 0 || n < 0 || lda < d || (n > 0 && !A))
+    return KRONQ_ERR_INVALID_ARG;
+  if (dtype != KRONQ_F32 && dtype != KRONQ_BF16) return KRONQ_ERR_INVALID_ARG;
+  if (d > (int64_t(1) << 20) || n > (int64_t(1) << 31)) return KRONQ_ERR_UNSUPPORTED;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  if (dtype == KRONQ_BF16) {
+    if (d % 128 || lda % 8 || !aligned(A, 16)) return KRONQ_ERR_UNSUPPORTED;
+    return cov_bf16(st, static_cast<const __nv_bfloat16 *>(A), n, d, lda, alpha,
+                    beta, H);
+  }
+  return cov_f32(st, static_cast<const float *>(A), n, d, lda, alpha, beta, H);
+}
+
+kronq_status kronq_sensitivity(kronq_stream_t stream, const float *H_X,
+                               int64_t d_in, const float *H_G, int64_t d_out,
+                               double *out_dev) {
+  if (!H_X || !H_G || !out_dev || d_in <= 0 || d_out <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  return launch_sensitivity(as_stream(stream), H_X, d_in, H_G, d_out, out_dev);
+}
+
+size_t kronq_workspace_bytes(kronq_ws_kind which, int64_t d_out, int64_t d_in,
+                             const kronq_opts *opts) {
+  if (d_out <= 0 || d_in <= 0) return 0;
+  switch (which) {
+    case KRONQ_WS_BIIP:
+      if (!opts || opts->rot_in.m < 1 || opts->rot_in.m > 256 ||
+          opts->rot_out.m < 1 || opts->rot_out.m > 256)
+        return 0;
+      return biip_ws_bytes(d_out, d_in, *opts);
+    case KRONQ_WS_CHOL:
+      if (d_in % 128) return 0;
+      return chol_ws_bytes(d_in);
+    case KRONQ_WS_QUANT:
+      if (!opts) return 0;
+      return quant_ws_bytes(d_out, d_in, *opts);
+    case KRONQ_WS_LOSS:
+      return loss_ws_bytes(d_out, d_in);
+  }
+  return 0;
+}
+
+kronq_status kronq_biip(kronq_stream_t stream, const kronq_opts *opts,
+                        const void *W, kronq_dtype wdtype, int64_t d_out,
+                        int64_t d_in, float *W_rot, float *H_X, float *H_G,
+                        float *s_x, float *s_g, void *ws, size_t ws_bytes,
+                        int32_t *info_dev) {
+  if (!opts || !W || !W_rot || !H_X || !H_G || !s_x || !s_g || !ws ||
+      !info_dev || d_out <= 0 || d_in <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  if (wdtype != KRONQ_F32 && wdtype != KRONQ_BF16) return KRONQ_ERR_INVALID_ARG;
+  if (!(opts->scale_exp >= 0.f && opts->scale_exp <= 4.f)) return KRONQ_ERR_INVALID_ARG;
+  const bool rot_x = !(opts->flags & KRONQ_FLAG_NO_ROT_IN);
+  const bool rot_g = !(opts->flags & KRONQ_FLAG_NO_ROT_OUT);
+  if (rot_x && !rot_ok(opts->rot_in, d_in)) return KRONQ_ERR_UNSUPPORTED;
+  if (rot_g && !rot_ok(opts->rot_out, d_out)) return KRONQ_ERR_UNSUPPORTED;
+  if (d_in % 32 || d_in > 65536 || d_out > 65536)
+    return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256)) return KRONQ_ERR_INVALID_ARG;
+  kronq_opts o = *opts;
+  if (!rot_x) o.rot_in = {d_in, 1};
+  if (!rot_g) o.rot_out = {d_out, 1};
+  if (ws_bytes < biip_ws_bytes(d_out, d_in, o)) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return biip(st, o, W, wdtype == KRONQ_BF16, d_out, d_in, W_rot, H_X, H_G, s_x,
+              s_g, ws, ws_bytes, info_dev);
+}
+
+kronq_status kronq_chol_inv(kronq_stream_t stream, float *H, int64_t d,
+                            float damp_rel, void *ws, size_t ws_bytes,
+                            int32_t *info_dev) {
+  if (!H || !ws || !info_dev || d <= 0 || !(damp_rel >= 0.f) || !isfinite(damp_rel))
+    return KRONQ_ERR_INVALID_ARG;
+  if (d % 128 || d > 65536) return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !aligned(H, 16)) return KRONQ_ERR_INVALID_ARG;
+  if (ws_bytes < chol_ws_bytes(d)) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return chol_inv(st, H, d, damp_rel, ws, ws_bytes, info_dev);
+}
+
+kronq_status kronq_quantize_sublayer(kronq_stream_t stream,
+                                     const kronq_opts *opts, float *W_rot,
+                                     const float *U, int64_t d_out,
+                                     int64_t d_in, uint32_t *codes,
+                                     float *scales, uint8_t *zeros, void *ws,
+                                     size_t ws_bytes, int32_t *info_dev) {
+  if (!opts || !W_rot || !U || !codes || !scales || !zeros || !ws ||
+      !info_dev || d_out <= 0 || d_in <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  if (opts->bits < 2 || opts->bits > 4) return KRONQ_ERR_INVALID_ARG;
+  if (opts->group != 32 && opts->group != 64 && opts->group != 128)
+    return KRONQ_ERR_UNSUPPORTED;
+  if (opts->block != 128 || d_in % 128) return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !aligned(W_rot, 16) || !aligned(U, 16))
+    return KRONQ_ERR_INVALID_ARG;
+  if (ws_bytes < quant_ws_bytes(d_out, d_in, *opts)) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return quantize(st, *opts, W_rot, U, d_out, d_in, codes, scales, zeros, ws,
+                  ws_bytes, info_dev);
+}
+
+kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
+                              const float *W_hat, const float *H_X,
+                              const float *H_G, int64_t d_out, int64_t d_in,
+                              double *loss_dev, void *ws, size_t ws_bytes) {
+  if (!W_ref || !W_hat || !H_X || !H_G || !loss_dev || !ws || d_out <= 0 ||
+      d_in <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  if (d_in % 128 || d_out % 128) return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !aligned(W_ref, 16) || !aligned(W_hat, 16) ||
+      !aligned(H_X, 16) || !aligned(H_G, 16))
+    return KRONQ_ERR_INVALID_ARG;
+  if (ws_bytes < loss_ws_bytes(d_out, d_in)) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  return layer_loss(as_stream(stream), W_ref, W_hat, H_X, H_G, d_out, d_in,
+                    loss_dev, ws, ws_bytes);
+}
+
+kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,
+                                 int n, double avg_budget, int *bits_out) {
+  if (!score || !numel || !bits_out || n <= 0 || !(avg_budget >= 2.0))
+    return KRONQ_ERR_INVALID_ARG;
+  double total = 0.0;
+  for (int i = 0; i < n; ++i) {
+    if (numel[i] <= 0 || !isfinite(score[i])) return KRONQ_ERR_INVALID_ARG;
+    total += static_cast<double>(numel[i]);
+  }
+  std::vector<int> order(n);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int b) { return score[a] > score[b]; });
+  for (int i = 0; i < n; ++i) bits_out[i] = 2;
+  double used = 2.0 * total;
+  const double cap = avg_budget * total;
+  for (int from = 2; from <= 3; ++from) {
+    for (int k = 0; k < n; ++k) {
+      const int i = order[k];
+      if (bits_out[i] == from && used + static_cast<double>(numel[i]) <= cap) {
+        bits_out[i] = from + 1;
+        used += static_cast<double>(numel[i]);
+      }
+    }
+  }
+  return KRONQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// Internal launcher interfaces between the C-ABI layer (api.cu) and the
+// kernels. Nothing here is exported.
+#pragma once
+
+#include "common.cuh"
+
+namespace kronq {
+
+// ---------------------------------------------------------------- GEMM
+// C = beta*C + alpha * A * B^T in fp32 with 3xTF32 tcgen05 MMAs.
+//   A is M x K: stored row-major (A[i*lda+k], K-major) or, with a_mn, as
+//   K x M (A[k*lda+i]). B is N x K: B[j*ldb+k], or with b_mn B[k*ldb+j].
+// Per-tile K ranges skip blocks that a triangular operand keeps at zero.
+enum : uint32_t {
+  KR_A_UPPER = 1u,  // A[i][k] == 0 for k < i  -> k starts at the tile's m0
+  KR_B_UPPER = 2u,  // B[j][k] == 0 for k < j  -> k starts at the tile's n0
+  KR_B_LOWER = 4u,  // B[j][k] == 0 for k > j  -> k ends at n0 + 128
+  KR_A_LOWER = 8u   // A[i][k] == 0 for k > i  -> k ends at m0 + 128
+};
+
+struct GemmArgs {
+  int64_t M = 0, N = 0, K = 0;
+  const float *A = nullptr;
+  int64_t lda = 0;
+  bool a_mn = false;
+  const float *B = nullptr;
+  int64_t ldb = 0;
+  bool b_mn = false;
+  float *C = nullptr;
+  int64_t ldc = 0;
+  float alpha = 1.f, beta = 0.f;
+  uint32_t kflags = 0;
+  bool upper_tiles_only = false;  // square C: only tiles with m0 <= n0
+};
+
+kronq_status gemm_tf32x3(cudaStream_t st, const GemmArgs &g, int32_t *info);
+
+// ---------------------------------------------------------------- covariance
+kronq_status cov_bf16(cudaStream_t st, const __nv_bfloat16 *A, int64_t n,
+                      int64_t d, int64_t lda, float alpha, float beta,
+                      float *H);
+kronq_status cov_f32(cudaStream_t st, const float *A, int64_t n, int64_t d,
+                     int64_t lda, float alpha, float beta, float *H);
+kronq_status scale_matrix(cudaStream_t st, float *H, int64_t n_elems,
+                          float beta);
+
+// ---------------------------------------------------------------- misc
+kronq_status launch_sensitivity(cudaStream_t st, const float *hx, int64_t dx,
+                                const float *hg, int64_t dg, double *out);
+kronq_status launch_set_int(cudaStream_t st, int32_t *p, int32_t v);
+
+// ---------------------------------------------------------------- Cholesky
+size_t chol_ws_bytes(int64_t d);
+kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
+                      void *ws, size_t ws_bytes, int32_t *info);
+
+// ---------------------------------------------------------------- BiIP
+size_t biip_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &o);
+kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
+                  bool w_bf16, int64_t d_out, int64_t d_in, float *W_rot,
+                  float *H_X, float *H_G, float *s_x, float *s_g, void *ws,
+                  size_t ws_bytes, int32_t *info);
+
+// ---------------------------------------------------------------- OBS
+size_t quant_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &o);
+kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
+                      const float *U, int64_t d_out, int64_t d_in,
+                      uint32_t *codes, float *scales, uint8_t *zeros,
+                      void *ws, size_t ws_bytes, int32_t *info);
+
+// ---------------------------------------------------------------- loss
+size_t loss_ws_bytes(int64_t d_out, int64_t d_in);
+kronq_status layer_loss(cudaStream_t st, const float *W_ref,
+                        const float *W_hat, const float *H_X, const float *H_G,
+                        int64_t d_out, int64_t d_in, double *loss, void *ws,
+                        size_t ws_bytes);
+
+}  // namespace kronq

@@ -1,0 +1,105 @@
+// Small helpers: device check, TMA tensor maps, sensitivity traces.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include "kernels.cuh"
+
+namespace kronq {
+namespace {
+
+__global__ void sensitivity_kernel(const float *hx, int64_t dx, const float *hg,
+                                   int64_t dg, double *out) {
+  __shared__ double part[2][32];
+  double sx = 0.0, sg = 0.0;
+  for (int64_t i = threadIdx.x; i < dx; i += blockDim.x) sx += hx[i * dx + i];
+  for (int64_t i = threadIdx.x; i < dg; i += blockDim.x) sg += hg[i * dg + i];
+  sx = warp_sum_d(sx);
+  sg = warp_sum_d(sg);
+  if ((threadIdx.x & 31) == 0) {
+    part[0][threadIdx.x >> 5] = sx;
+    part[1][threadIdx.x >> 5] = sg;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0, b = 0.0;
+    for (int k = 0; k < int(blockDim.x / 32); ++k) {
+      a += part[0][k];
+      b += part[1][k];
+    }
+    out[0] = a;
+    out[1] = b;
+    out[2] = a * b;
+  }
+}
+
+__global__ void set_int_kernel(int32_t *p, int32_t v) { *p = v; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
+                                &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+kronq_status require_sm100() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KRONQ_ERR_CUDA;
+  static int checked_dev = -1;
+  static bool ok = false;
+  if (checked_dev != dev) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    ok = (major == 10 && minor == 0);
+    checked_dev = dev;
+  }
+  return ok ? KRONQ_OK : KRONQ_ERR_CUDA;
+}
+
+kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
+                          uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+                          uint32_t box_inner, uint32_t box_outer,
+                          bool swz32) {
+  const uint64_t es = bf16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0) return KRONQ_ERR_UNSUPPORTED;
+  if ((pitch_elems * es) % 16 != 0) return KRONQ_ERR_UNSUPPORTED;
+  auto fn = encode_fn();
+  if (!fn) return KRONQ_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * es};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map,
+                  bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? KRONQ_OK : KRONQ_ERR_CUDA;
+}
+
+kronq_status launch_sensitivity(cudaStream_t st, const float *hx, int64_t dx,
+                                const float *hg, int64_t dg, double *out) {
+  sensitivity_kernel<<<1, 1024, 0, st>>>(hx, dx, hg, dg, out);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+kronq_status launch_set_int(cudaStream_t st, int32_t *p, int32_t v) {
+  set_int_kernel<<<1, 1, 0, st>>>(p, v);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+}  // namespace kronq

@@ -1,0 +1,186 @@
+// Blocked column-wise OBS quantize-and-compensate [gptget-en Methodology:
+// extends GPTQ's column-wise OBS; wmrh §四: the per-column update is GPTAQ's
+// and H_G does not enter it, so rows are independent given U; wmrh §五:
+// W2/W3/W4 with 128-column groups].
+//
+// Per 128-column block j0 (one launch of obs_block_kernel): each warp owns one
+// row at a time, the block's 128 weights of the row live in 4 registers per
+// lane, U[j0:j0+128, j0:j0+128] sits in shared memory. For each column j:
+// group (scale, zero) at a group start, q = clamp(rint(w/scale)+zero),
+// err = (w - w_hat)/U[j][j], w_k -= err * U[j][k] for the block's k > j.
+// The errors go to E; the columns right of the block are updated lazily by
+// 3xTF32 GEMMs: within a super-block of S columns after every block
+// (W[:, blk_end:sb_end] -= E_blk U[blk, blk_end:sb_end]), and once per
+// super-block for everything right of it (W[:, sb_end:] -= E_sb U[sb, sb_end:]).
+// Codes are packed in the same pass (little-endian bitstream per row).
+#include "kernels.cuh"
+
+namespace kronq {
+namespace {
+
+constexpr int OB = 128;        // block width
+constexpr int OTHREADS = 512;  // 16 warps
+constexpr int ROWS_PER_WARP = 4;
+constexpr int OROWS = (OTHREADS / 32) * ROWS_PER_WARP;
+constexpr int SUPER = 1024;    // super-block width
+
+__device__ __forceinline__ float pick4(const float (&v)[4], int s) {
+  return s == 0 ? v[0] : s == 1 ? v[1] : s == 2 ? v[2] : v[3];
+}
+
+__global__ void __launch_bounds__(OTHREADS)
+    obs_block_kernel(float *__restrict__ W, int64_t ldw,
+                     const float *__restrict__ U, int64_t ldu, int64_t j0,
+                     int64_t d_out, int bits, int group,
+                     float *__restrict__ E, int64_t lde, int64_t e_col,
+                     uint32_t *__restrict__ codes, int64_t ldq,
+                     float *__restrict__ scales, uint8_t *__restrict__ zeros,
+                     int64_t ngroups) {
+  extern __shared__ float Us[];                      // OB x OB
+  __shared__ uint8_t qsm[OTHREADS / 32][OB];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < OB * OB; e += OTHREADS) {
+    const int r = e / OB, c = e % OB;
+    Us[e] = U[(j0 + r) * ldu + j0 + c];
+  }
+  __syncthreads();
+  const float maxq = static_cast<float>((1 << bits) - 1);
+  for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
+    const int64_t row =
+        int64_t(blockIdx.x) * OROWS + warp * ROWS_PER_WARP + rr;
+    if (row >= d_out) break;
+    float w[4], err[4], qv[4];
+    float *wrow = W + row * ldw + j0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      w[s] = wrow[lane + 32 * s];
+      err[s] = 0.f;
+      qv[s] = 0.f;
+    }
+    float scale = 1.f, zero = 0.f;
+    for (int j = 0; j < OB; ++j) {
+      if (j % group == 0) {
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int c = lane + 32 * s;
+          if (c >= j && c < j + group) {
+            mn = fminf(mn, w[s]);
+            mx = fmaxf(mx, w[s]);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        const float xmin = fminf(mn, 0.f), xmax = fmaxf(mx, 0.f);
+        if (xmax == xmin) {
+          scale = 1.f;
+          zero = 0.f;
+        } else {
+          scale = (xmax - xmin) / maxq;
+          zero = rintf(-xmin / scale);
+        }
+        if (lane == 0) {
+          const int64_t gi = (j0 + j) / group;
+          scales[row * ngroups + gi] = scale;
+          zeros[row * ngroups + gi] = static_cast<uint8_t>(zero);
+        }
+      }
+      const int slot = j >> 5, owner = j & 31;
+      const float wj = __shfl_sync(0xffffffffu, pick4(w, slot), owner);
+      const float q = fminf(fmaxf(rintf(wj / scale) + zero, 0.f), maxq);
+      const float wh = scale * (q - zero);
+      const float e = (wj - wh) / Us[j * OB + j];
+      const float *urow = Us + j * OB;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int c = lane + 32 * s;
+        if (c > j) w[s] = fmaf(-e, urow[c], w[s]);
+        if (s == slot && lane == owner) {
+          w[s] = wh;
+          err[s] = e;
+          qv[s] = q;
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      wrow[lane + 32 * s] = w[s];
+      E[row * lde + e_col + lane + 32 * s] = err[s];
+      qsm[warp][lane + 32 * s] = static_cast<uint8_t>(qv[s]);
+    }
+    __syncwarp();
+    const int nwords = OB * bits / 32;
+    if (lane < nwords) {
+      uint32_t word = 0;
+      const int bit0 = 32 * lane;
+      const int c_lo = bit0 / bits, c_hi = min(OB - 1, (bit0 + 31) / bits);
+      for (int c = c_lo; c <= c_hi; ++c) {
+        const int sh = c * bits - bit0;
+        const uint32_t code = qsm[warp][c];
+        word |= sh >= 0 ? (code << sh) : (code >> (-sh));
+      }
+      codes[row * ldq + (j0 * bits) / 32 + lane] = word;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+size_t quant_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &) {
+  const int64_t S = kq_min<int64_t>(d_in, SUPER);
+  return static_cast<size_t>(d_out) * S * 4 + 256;
+}
+
+kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
+                      const float *U, int64_t d_out, int64_t d_in,
+                      uint32_t *codes, float *scales, uint8_t *zeros,
+                      void *ws, size_t ws_bytes, int32_t *info) {
+  if (ws_bytes < quant_ws_bytes(d_out, d_in, o)) return KRONQ_ERR_INVALID_ARG;
+  const int64_t S = kq_min<int64_t>(d_in, SUPER);
+  float *E = static_cast<float *>(ws);
+  const int64_t ngroups = d_in / o.group;
+  const int64_t ldq = o.bits * d_in / 32;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(obs_block_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             OB * OB * 4) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    attr_done = true;
+  }
+  const unsigned grid = static_cast<unsigned>(ceil_div(d_out, OROWS));
+  for (int64_t sb0 = 0; sb0 < d_in; sb0 += S) {
+    const int64_t sb1 = kq_min<int64_t>(d_in, sb0 + S);
+    for (int64_t j0 = sb0; j0 < sb1; j0 += OB) {
+      obs_block_kernel<<<grid, OTHREADS, OB * OB * 4, st>>>(
+          W, d_in, U, d_in, j0, d_out, o.bits, o.group, E, S, j0 - sb0, codes,
+          ldq, scales, zeros, ngroups);
+      KQ_CHECK_LAUNCH();
+      if (j0 + OB < sb1) {
+        GemmArgs g;
+        g.M = d_out; g.N = sb1 - j0 - OB; g.K = OB;
+        g.A = E + (j0 - sb0); g.lda = S;
+        g.B = U + j0 * d_in + j0 + OB; g.ldb = d_in; g.b_mn = true;
+        g.C = W + j0 + OB; g.ldc = d_in;
+        g.alpha = -1.f; g.beta = 1.f;
+        KQ_TRY(gemm_tf32x3(st, g, info));
+      }
+    }
+    if (sb1 < d_in) {
+      GemmArgs g;
+      g.M = d_out; g.N = d_in - sb1; g.K = sb1 - sb0;
+      g.A = E; g.lda = S;
+      g.B = U + sb0 * d_in + sb1; g.ldb = d_in; g.b_mn = true;
+      g.C = W + sb1; g.ldc = d_in;
+      g.alpha = -1.f; g.beta = 1.f;
+      KQ_TRY(gemm_tf32x3(st, g, info));
+    }
+  }
+  return KRONQ_OK;
+}
+
+}  // namespace kronq

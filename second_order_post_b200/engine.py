@@ -1,0 +1,91 @@
+"""One-sublayer KronQ quantization on the GPU through libkronq's C ABI.
+
+``SublayerEngine`` owns the device buffers (allocated once with torch, reused
+across calls) and enqueues the five steps on one CUDA stream:
+
+  1. kronq_accum_cov(X) -> H_X,  kronq_accum_cov(G) -> H_G
+  2. kronq_sensitivity(H_X, H_G)            (before the rotation)
+  3. kronq_biip -> W', H_X', H_G', s_x, s_g
+  4. kronq_chol_inv(H_X') -> U               (in place)
+  5. kronq_quantize_sublayer(W', U) -> codes, scales, zeros, W_hat (in place)
+
+All arithmetic runs in the library's kernels; this module only allocates and
+passes pointers.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import kronq as K
+
+
+@dataclasses.dataclass
+class QuantResult:
+    codes: torch.Tensor      # d_out x bits*d_in/32 uint32 words (int32 view)
+    scales: torch.Tensor     # d_out x d_in/group fp32
+    zeros: torch.Tensor      # d_out x d_in/group uint8
+    w_hat: torch.Tensor      # dequantized W' (rotated basis)
+    s_x: torch.Tensor
+    s_g: torch.Tensor
+    sens: torch.Tensor       # float64[3]: tr H_X, tr H_G, product
+
+
+class SublayerEngine:
+    def __init__(self, d_out, d_in, bits=4, group=128, damp_rel=0.01,
+                 scale_exp=0.25, seed=0, rot_in=None, rot_out=None, flags=0,
+                 device="cuda", keep_w_rot=False):
+        self.d_out, self.d_in = d_out, d_in
+        self.opts = K.make_opts(bits=bits, group=group, damp_rel=damp_rel,
+                                scale_exp=scale_exp, seed=seed,
+                                rot_in=rot_in or (d_in, 1),
+                                rot_out=rot_out or (d_out, 1), flags=flags)
+        dev = torch.device(device)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.H_X = torch.empty(d_in, d_in, **f32)
+        self.H_G = torch.empty(d_out, d_out, **f32)
+        self.W_rot = torch.empty(d_out, d_in, **f32)
+        self.W_ref = torch.empty(d_out, d_in, **f32) if keep_w_rot else None
+        self.s_x = torch.empty(d_in, **f32)
+        self.s_g = torch.empty(d_out, **f32)
+        self.sens = torch.zeros(3, dtype=torch.float64, device=dev)
+        ng = d_in // group
+        self.codes = torch.empty(d_out, bits * d_in // 32, dtype=torch.int32, device=dev)
+        self.scales = torch.empty(d_out, ng, **f32)
+        self.zeros = torch.empty(d_out, ng, dtype=torch.uint8, device=dev)
+        self.info = torch.zeros(3, dtype=torch.int32, device=dev)
+        ws = max(K.kronq_workspace_bytes(K.KRONQ_WS_BIIP, d_out, d_in, self.opts),
+                 K.kronq_workspace_bytes(K.KRONQ_WS_CHOL, d_out, d_in, self.opts),
+                 K.kronq_workspace_bytes(K.KRONQ_WS_QUANT, d_out, d_in, self.opts))
+        if ws == 0:
+            raise ValueError("unsupported sublayer shape for libkronq")
+        self.ws = torch.empty((ws + 255) // 256 * 256, dtype=torch.uint8, device=dev)
+
+    def covariances(self, X, G, stream=None):
+        K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, stream)
+        K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, stream)
+
+    def run(self, W, X, G, stream=None) -> QuantResult:
+        """Enqueue the whole sublayer quantization (no host synchronisation)."""
+        self.covariances(X, G, stream)
+        K.kronq_sensitivity(self.H_X, self.H_G, self.sens, stream)
+        K.kronq_biip(self.opts, W, self.W_rot, self.H_X, self.H_G, self.s_x,
+                     self.s_g, self.ws, self.info[0:1], stream)
+        if self.W_ref is not None:
+            self.W_ref.copy_(self.W_rot)
+        K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[1:2],
+                         stream)
+        K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, self.codes,
+                                  self.scales, self.zeros, self.ws,
+                                  self.info[2:3], stream)
+        return QuantResult(self.codes, self.scales, self.zeros, self.W_rot,
+                           self.s_x, self.s_g, self.sens)
+
+    def check_info(self):
+        """Raises KronqError for a non-zero device status word (syncs)."""
+        vals = self.info.tolist()
+        for name, v in zip(("kronq_biip", "kronq_chol_inv",
+                            "kronq_quantize_sublayer"), vals):
+            if v != 0:
+                raise K.KronqError(name, v & 0xFF)
