@@ -258,6 +258,11 @@ kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,
 /* Static, human-readable name of a status code. */
 const char *kronq_status_string(kronq_status s);
 
+/* Diagnostics (no counterpart on the pages): the number of CUDA kernels this
+ * process has launched through the library since it was loaded. Host call,
+ * thread-safe, never fails. */
+uint64_t kronq_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -196,4 +196,6 @@ kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,
   return KRONQ_OK;
 }
 
+uint64_t kronq_kernel_launches(void) { return launches(); }
+
 }  // extern "C"

@@ -17,8 +17,12 @@ template <class T>
 __host__ __device__ __forceinline__ T kq_max(T a, T b) { return a < b ? b : a; }
 
 // ----------------------------------------------------------------- host side
+// Counts every kernel the library launches (reported by kronq_kernel_launches).
+void count_launch();
+
 #define KQ_CHECK_LAUNCH()                                                      \
   do {                                                                         \
+    count_launch();                                                            \
     cudaError_t e_ = cudaGetLastError();                                       \
     if (e_ != cudaSuccess) return KRONQ_ERR_CUDA;                              \
   } while (0)

@@ -48,6 +48,7 @@ kronq_status scale_matrix(cudaStream_t st, float *H, int64_t n_elems,
 kronq_status launch_sensitivity(cudaStream_t st, const float *hx, int64_t dx,
                                 const float *hg, int64_t dg, double *out);
 kronq_status launch_set_int(cudaStream_t st, int32_t *p, int32_t v);
+uint64_t launches();
 
 // ---------------------------------------------------------------- Cholesky
 size_t chol_ws_bytes(int64_t d);

@@ -2,6 +2,8 @@
 #include <cudaTypedefs.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "kernels.cuh"
 
 namespace kronq {
@@ -49,6 +51,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 }  // namespace
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
 kronq_status require_sm100() {
   int dev = -1;

@@ -66,19 +66,28 @@ class SublayerEngine:
         K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, stream)
         K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, stream)
 
-    def run(self, W, X, G, stream=None) -> QuantResult:
-        """Enqueue the whole sublayer quantization (no host synchronisation)."""
-        self.covariances(X, G, stream)
+    def run(self, W, X, G, stream=None, mark=None) -> QuantResult:
+        """Enqueue the whole sublayer quantization (no host synchronisation).
+        ``mark(name)``, if given, is called after each step is enqueued (the
+        benchmark records a CUDA event there)."""
+        mark = mark or (lambda name: None)
+        K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, stream)
+        mark("cov_x")
+        K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, stream)
+        mark("cov_g")
         K.kronq_sensitivity(self.H_X, self.H_G, self.sens, stream)
         K.kronq_biip(self.opts, W, self.W_rot, self.H_X, self.H_G, self.s_x,
                      self.s_g, self.ws, self.info[0:1], stream)
+        mark("biip")
         if self.W_ref is not None:
             self.W_ref.copy_(self.W_rot)
         K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[1:2],
                          stream)
+        mark("chol")
         K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, self.codes,
                                   self.scales, self.zeros, self.ws,
                                   self.info[2:3], stream)
+        mark("quant")
         return QuantResult(self.codes, self.scales, self.zeros, self.W_rot,
                            self.s_x, self.s_g, self.sens)
 

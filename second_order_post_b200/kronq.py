@@ -79,6 +79,7 @@ _SIGS = {
     "kronq_workspace_bytes": [ctypes.c_int, _i64, _i64, _OPTS],
     "kronq_allocate_bits": [_p, _p, ctypes.c_int, _d, _p],
     "kronq_status_string": [ctypes.c_int],
+    "kronq_kernel_launches": [],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -86,6 +87,7 @@ for _name, _args in _SIGS.items():
     _fn.restype = ctypes.c_int
 _lib.kronq_workspace_bytes.restype = ctypes.c_size_t
 _lib.kronq_status_string.restype = ctypes.c_char_p
+_lib.kronq_kernel_launches.restype = ctypes.c_uint64
 
 
 def _check(fn, st):
@@ -176,6 +178,11 @@ def kronq_allocate_bits(scores, numel, avg_budget):
 
 def kronq_status_string(status):
     return _lib.kronq_status_string(status).decode()
+
+
+def kronq_kernel_launches():
+    """Kernels this process has launched through the library so far."""
+    return int(_lib.kronq_kernel_launches())
 
 
 def exported_symbols():
