@@ -200,6 +200,35 @@ kronq_status kronq_biip(kronq_stream_t stream, const kronq_opts *opts,
                         int32_t *info_dev);
 
 /*
+ * Step 3 for callers that cannot allocate device memory. The pages have no
+ * counterpart: this is a deployment convenience, not part of the method.
+ * Some callers cannot give the library a workspace: frameworks that reserve
+ * all of HBM for their own pool allocator, plugin hosts that pass only
+ * input and output buffers, or loops where cudaMalloc/cudaFree would
+ * synchronise the device. This call behaves exactly like kronq_biip (same
+ * arguments without ws/ws_bytes, same results, errors and info word) but
+ * keeps its scratch in a fixed 4 MiB device array inside the library. It
+ * calls no allocator.
+ * - The array lives in the module image: every GPU that loads libkronq.so
+ *   holds 4 MiB for it until the process exits.
+ * - The first call on a device looks up the array's device address, with
+ *   that device current, and caches it. Make that first call before any
+ *   stream capture on the device.
+ * - All calls share the one array. It keeps the last call's contents, but
+ *   nothing in it has to start at zero: every byte a call reads is written
+ *   earlier in the same call.
+ * - Calls that overlap on the GPU (other streams, other host threads) race
+ *   on the array. Serialise them.
+ * - Sizes whose scratch would not fit return KRONQ_ERR_UNSUPPORTED. Every
+ *   size that kronq_biip accepts (d <= 65536, m <= 256) fits.
+ */
+kronq_status kronq_biip_noalloc(kronq_stream_t stream, const kronq_opts *opts,
+                                const void *W, kronq_dtype wdtype,
+                                int64_t d_out, int64_t d_in, float *W_rot,
+                                float *H_X, float *H_G, float *s_x, float *s_g,
+                                int32_t *info_dev);
+
+/*
  * Step 4 — damped inverse Cholesky factor [wmrh §四; GPTQ-style OBS needs
  * the upper factor of the inverse Hessian].
  * In: H (d x d fp32, full symmetric, e.g. H_X'). Out, in place: U upper

@@ -72,6 +72,8 @@ _SIGS = {
     "kronq_sensitivity": [_p, _p, _i64, _p, _i64, _p],
     "kronq_biip": [_p, _OPTS, _p, ctypes.c_int, _i64, _i64, _p, _p, _p, _p, _p,
                    _p, _sz, _p],
+    "kronq_biip_noalloc": [_p, _OPTS, _p, ctypes.c_int, _i64, _i64, _p, _p, _p,
+                           _p, _p, _p],
     "kronq_chol_inv": [_p, _p, _i64, _f, _p, _sz, _p],
     "kronq_quantize_sublayer": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p,
                                 _sz, _p],
@@ -140,6 +142,16 @@ def kronq_biip(opts, W, W_rot, H_X, H_G, s_x, s_g, ws, info, stream=None):
         _stream(stream), ctypes.byref(opts), _ptr(W), _dtype(W), d_out, d_in,
         _ptr(W_rot), _ptr(H_X), _ptr(H_G), _ptr(s_x), _ptr(s_g), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(info)))
+
+
+def kronq_biip_noalloc(opts, W, W_rot, H_X, H_G, s_x, s_g, info, stream=None):
+    """kronq_biip without a workspace, for callers that cannot allocate device
+    memory; the library's own fixed device array serves as scratch (calls
+    that overlap on the GPU race on it)."""
+    d_out, d_in = W.shape
+    _check("kronq_biip_noalloc", _lib.kronq_biip_noalloc(
+        _stream(stream), ctypes.byref(opts), _ptr(W), _dtype(W), d_out, d_in,
+        _ptr(W_rot), _ptr(H_X), _ptr(H_G), _ptr(s_x), _ptr(s_g), _ptr(info)))
 
 
 def kronq_chol_inv(H, damp_rel, ws, info, stream=None):
