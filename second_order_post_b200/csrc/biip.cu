@@ -22,9 +22,6 @@
 namespace kronq {
 namespace {
 
-constexpr int TILE_BUDGET = 12288;   // floats per tile buffer
-constexpr int SLAB_BUDGET = 32768;   // floats per strided slab
-constexpr int MAX_A = 1024;          // Hadamard length of one strided pass
 
 __host__ __device__ inline uint64_t sm64(uint64_t s) {
   uint64_t z = s + 0x9E3779B97F4A7C15ull;
@@ -149,145 +146,203 @@ __global__ void qm_kernel(QDev a, QDev b) {
   }
 }
 
-// ------------------------------------------------------------- tile pass
-struct TileP {
+// ------------------------------------------------------------- Hadamard helpers
+// In-register Hadamard of R values (unnormalised).
+template <int R>
+__device__ __forceinline__ void fwht_reg(float (&r)[R]) {
+#pragma unroll
+  for (int s = 1; s < R; s <<= 1)
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      if (!(i & s)) {
+        const float u = r[i], w = r[i + s];
+        r[i] = u + w;
+        r[i + s] = u - w;
+      }
+}
+
+// One radix-R round of a length-L Hadamard over n_vec vectors held in shared
+// memory (element j of vector v at X[vbase(v) + j*stride]): combines the R
+// elements a + i*h, i < R, for every a whose index bits h .. R*h-1 are clear.
+template <int R, class VB>
+__device__ void fwht_round(float *X, int n_vec, int L, int h, int stride, VB vbase) {
+  const int groups = L / R;
+  for (int idx = threadIdx.x; idx < groups * n_vec; idx += blockDim.x) {
+    const int v = idx % n_vec, g = idx / n_vec;
+    const int a = (g / h) * R * h + (g % h);
+    float *x = X + vbase(v) + a * stride;
+    float r[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) r[i] = x[i * h * stride];
+    fwht_reg<R>(r);
+#pragma unroll
+    for (int i = 0; i < R; ++i) x[i * h * stride] = r[i];
+  }
+  __syncthreads();
+}
+
+// Remaining rounds of a length-L Hadamard whose distances below h are done.
+template <class VB>
+__device__ void fwht_rest(float *X, int n_vec, int L, int h, int stride, VB vbase) {
+  while (h * 16 <= L) {
+    fwht_round<16>(X, n_vec, L, h, stride, vbase);
+    h *= 16;
+  }
+  const int rem = L / h;
+  if (rem == 2) fwht_round<2>(X, n_vec, L, h, stride, vbase);
+  else if (rem == 4) fwht_round<4>(X, n_vec, L, h, stride, vbase);
+  else if (rem == 8) fwht_round<8>(X, n_vec, L, h, stride, vbase);
+}
+
+// ------------------------------------------------------------- row pass
+// One CTA per (row, chunk of L*m contiguous columns) of an R x C matrix:
+// out = norm * cr[row] * (Hhat_L ⊗ Q_m)(cc ⊙ x) on the chunk. The chunk lives
+// in shared memory (element a*m + b); the first radix-16 Hadamard round runs
+// in registers while loading, the Q_m mix runs while storing.
+struct RowP {
   const void *in;
   float *out;
   int64_t ld_in, ld_out;
   int in_bf16;
-  const float *cr, *cc;  // row / column factors (null = 1)
+  const float *cr, *cc;
   float norm;
-  int kr, Lr, mr;        // tile rows = kr * Lr * mr
-  int kc, Lc, mc;        // tile cols = kc * Lc * mc
-  const float *Qr, *Qc;  // Q_m of the row side / column side (null = skip)
-  int64_t tiles_c;
+  int L, m;
+  const float *Q;  // m x m row-major, null when m == 1
+  int64_t chunks;  // chunks per row
 };
 
-__device__ __forceinline__ float ld_in(const TileP &p, int64_t off) {
-  return p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.in)[off])
-                   : reinterpret_cast<const float *>(p.in)[off];
+__device__ __forceinline__ float load_in(const void *p, int bf16, int64_t off) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[off])
+              : reinterpret_cast<const float *>(p)[off];
 }
 
-// Radix-2 Hadamard butterflies over n_vec vectors of length L; element j of
-// vector v lives at base(v) + j*stride.
-template <class Base>
-__device__ void fwht_smem(float *X, int n_vec, int L, int stride, Base base) {
-  for (int h = 1; h < L; h <<= 1) {
-    const int half = L >> 1;
-    const int total = n_vec * half;
-    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-      const int v = idx % n_vec, pidx = idx / n_vec;
-      const int a = (pidx / h) * 2 * h + (pidx % h);
-      float *x = X + base(v) + a * stride;
-      const float u = x[0], w = x[h * stride];
-      x[0] = u + w;
-      x[h * stride] = u - w;
+template <int R0>
+__device__ void row_load_round(const RowP &p, float *X, int64_t row, int64_t c0) {
+  const int m = p.m, L = p.L;
+  const float rf = p.norm * (p.cr ? p.cr[row] : 1.f);
+  const int groups = L / R0;
+  for (int idx = threadIdx.x; idx < groups * m; idx += blockDim.x) {
+    const int b = idx % m, g = idx / m;
+    float r[R0];
+#pragma unroll
+    for (int i = 0; i < R0; ++i) {
+      const int e = (g * R0 + i) * m + b;
+      float v = load_in(p.in, p.in_bf16, row * p.ld_in + c0 + e) * rf;
+      if (p.cc) v *= p.cc[c0 + e];
+      r[i] = v;
+    }
+    fwht_reg<R0>(r);
+#pragma unroll
+    for (int i = 0; i < R0; ++i) X[(g * R0 + i) * m + b] = r[i];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(512) row_pass_kernel(RowP p) {
+  extern __shared__ float X[];
+  const int m = p.m, L = p.L, chunk = L * m;
+  const int64_t row = blockIdx.x / p.chunks;
+  const int64_t c0 = (blockIdx.x % p.chunks) * int64_t(chunk);
+  auto vb = [=](int v) { return v; };
+  int h;
+  if (L >= 16) {
+    row_load_round<16>(p, X, row, c0);
+    h = 16;
+  } else if (L == 8) {
+    row_load_round<8>(p, X, row, c0);
+    h = 8;
+  } else if (L == 4) {
+    row_load_round<4>(p, X, row, c0);
+    h = 4;
+  } else if (L == 2) {
+    row_load_round<2>(p, X, row, c0);
+    h = 2;
+  } else {
+    row_load_round<1>(p, X, row, c0);
+    h = 1;
+  }
+  fwht_rest(X, m, L, h, m, vb);
+  float *o = p.out + row * p.ld_out + c0;
+  if (p.Q == nullptr) {
+    for (int e = threadIdx.x; e < chunk; e += blockDim.x) o[e] = X[e];
+    return;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (m <= 32) {
+    // lane b owns output b of every group; its row of Q_m stays in registers
+    float q[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) q[k] = (lane < m && k < m) ? p.Q[lane * m + k] : 0.f;
+    for (int a = warp; a < L; a += nw) {
+      const float *x = X + a * m;
+      float y = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        if (k < m) y = fmaf(q[k], x[k], y);
+      if (lane < m) o[a * m + lane] = y;
+    }
+  } else {
+    // lanes own outputs b = lane + 32j; Q_m read from global (cached)
+    for (int a = warp; a < L; a += nw) {
+      const float *x = X + a * m;
+      for (int b = lane; b < m; b += 32) {
+        const float *qr = p.Q + b * m;
+        float y = 0.f;
+        for (int k = 0; k < m; ++k) y = fmaf(__ldg(qr + k), x[k], y);
+        o[a * m + b] = y;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- row-side Q_m
+// out[(a*m + b)][c] = sum_k Q[b][k] * in[(a*m + k)][c] for groups of m
+// consecutive rows; one thread per column, in place.
+__global__ void __launch_bounds__(256)
+    rowq_kernel(float *M, int64_t ld, int64_t C, int m, const float *Q) {
+  extern __shared__ float sm[];  // Q (m*m), then a [m][64] tile when m > 32
+  for (int e = threadIdx.x; e < m * m; e += blockDim.x) sm[e] = Q[e];
+  __syncthreads();
+  const int64_t a = blockIdx.y;
+  float *base = M + a * m * ld;
+  if (m <= 32) {
+    const int64_t c = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (c >= C) return;
+    float x[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) x[k] = k < m ? base[k * ld + c] : 0.f;
+    for (int b = 0; b < m; ++b) {
+      const float *qr = sm + b * m;
+      float y = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        if (k < m) y = fmaf(qr[k], x[k], y);
+      base[b * ld + c] = y;
+    }
+  } else {
+    float *T = sm + m * m;  // [m][64]
+    const int64_t c0 = blockIdx.x * int64_t(64);
+    for (int e = threadIdx.x; e < m * 64; e += blockDim.x) {
+      const int k = e / 64, c = e % 64;
+      T[e] = (c0 + c < C) ? base[k * ld + c0 + c] : 0.f;
     }
     __syncthreads();
-  }
-}
-
-// y = Q x for n_vec vectors of length m (element b at base(v) + b*stride);
-// output written to Y at the same positions. Four outputs per thread.
-template <class Base>
-__device__ void qmix_smem(const float *X, float *Y, const float *Q, int n_vec,
-                          int m, int stride, Base base) {
-  const int nb4 = (m + 3) / 4;
-  const int total = n_vec * nb4;
-  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-    const int v = idx % n_vec, b0 = (idx / n_vec) * 4;
-    const int bo = base(v);
-    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-    const float *q0 = Q + b0 * m;
-    for (int k = 0; k < m; ++k) {
-      const float x = X[bo + k * stride];
-      y0 = fmaf(q0[k], x, y0);
-      if (b0 + 1 < m) y1 = fmaf(q0[m + k], x, y1);
-      if (b0 + 2 < m) y2 = fmaf(q0[2 * m + k], x, y2);
-      if (b0 + 3 < m) y3 = fmaf(q0[3 * m + k], x, y3);
+    const int c = threadIdx.x % 64, bq = threadIdx.x / 64;
+    if (c0 + c < C) {
+      for (int b = bq; b < m; b += blockDim.x / 64) {
+        const float *qr = sm + b * m;
+        float y = 0.f;
+        for (int k = 0; k < m; ++k) y = fmaf(qr[k], T[k * 64 + c], y);
+        base[b * ld + c0 + c] = y;
+      }
     }
-    Y[bo + b0 * stride] = y0;
-    if (b0 + 1 < m) Y[bo + (b0 + 1) * stride] = y1;
-    if (b0 + 2 < m) Y[bo + (b0 + 2) * stride] = y2;
-    if (b0 + 3 < m) Y[bo + (b0 + 3) * stride] = y3;
-  }
-  __syncthreads();
-}
-
-__global__ void __launch_bounds__(512) tile_pass_kernel(TileP p) {
-  extern __shared__ float sm[];
-  const int TR = p.kr * p.Lr * p.mr, TC = p.kc * p.Lc * p.mc;
-  const int TCP = TC + ((TC & 1) ? 0 : 1);
-  const bool stage = (p.Qr != nullptr) || (p.Qc != nullptr);
-  float *T = sm;
-  float *S = sm + TR * TCP;
-  float *qsm = stage ? S + TR * TCP : sm + TR * TCP;
-  const float *Qr = p.Qr, *Qc = p.Qc;
-  // small Q_m into shared memory
-  {
-    float *q = qsm;
-    if (p.Qc && p.mc * p.mc <= 4096) {
-      for (int e = threadIdx.x; e < p.mc * p.mc; e += blockDim.x) q[e] = p.Qc[e];
-      Qc = q;
-      q += p.mc * p.mc;
-    }
-    if (p.Qr && p.mr * p.mr <= 4096) {
-      for (int e = threadIdx.x; e < p.mr * p.mr; e += blockDim.x) q[e] = p.Qr[e];
-      Qr = q;
-    }
-  }
-  const int64_t tr = blockIdx.x / p.tiles_c, tc = blockIdx.x % p.tiles_c;
-  const int64_t r0 = tr * TR, c0 = tc * TC;
-  for (int e = threadIdx.x; e < TR * TC; e += blockDim.x) {
-    const int r = e / TC, c = e % TC;
-    float v = ld_in(p, (r0 + r) * p.ld_in + c0 + c) * p.norm;
-    if (p.cr) v *= p.cr[r0 + r];
-    if (p.cc) v *= p.cc[c0 + c];
-    T[r * TCP + c] = v;
-  }
-  __syncthreads();
-  // ---- column side (within each row): Hadamard over a'_lo, then Q_c over b'
-  const int Lc = p.Lc, mc = p.mc, Lr = p.Lr, mr = p.mr;
-  if (Lc > 1) {
-    const int nv = TR * p.kc * mc;
-    fwht_smem(T, nv, Lc, mc, [=](int v) {
-      const int b = v % mc, t2 = v / mc, kb = t2 % p.kc, r = t2 / p.kc;
-      return r * TCP + kb * Lc * mc + b;
-    });
-  }
-  if (Qc) {
-    const int nv = TR * p.kc * Lc;
-    qmix_smem(T, S, Qc, nv, mc, 1, [=](int v) {
-      const int r = v % TR, g = v / TR;  // g = kb*Lc + a
-      return r * TCP + g * mc;
-    });
-    float *t = T; T = S; S = t;
-  }
-  // ---- row side (across rows): Hadamard over a_lo, then Q_r over b
-  if (Lr > 1) {
-    const int nv = TC * p.kr * mr;
-    fwht_smem(T, nv, Lr, mr * TCP, [=](int v) {
-      const int c = v % TC, t2 = v / TC, b = t2 % mr, kb = t2 / mr;
-      return (kb * Lr * mr + b) * TCP + c;
-    });
-  }
-  if (Qr) {
-    const int nv = TC * p.kr * Lr;
-    qmix_smem(T, S, Qr, nv, mr, TCP, [=](int v) {
-      const int c = v % TC, g = v / TC;  // g = kb*Lr + a
-      return g * mr * TCP + c;
-    });
-    float *t = T; T = S; S = t;
-  }
-  for (int e = threadIdx.x; e < TR * TC; e += blockDim.x) {
-    const int r = e / TC, c = e % TC;
-    p.out[(r0 + r) * p.ld_out + c0 + c] = T[r * TCP + c];
   }
 }
 
 // ------------------------------------------------------------- strided pass
-// View [outer][A][inner] at strides (so, sm, 1); Hadamard (unnormalised) of
-// length A along the middle axis; one [A][cw] slab per CTA.
+// View [outer][A][inner] at strides (so, smid, 1); Hadamard (unnormalised) of
+// length A along the middle axis; one [A][cw] slab per CTA, first radix-16
+// round in registers while loading.
 __global__ void __launch_bounds__(512)
     strided_fwht_kernel(float *base, int64_t so, int A, int64_t smid,
                         int64_t inner, int cw, int64_t chunks) {
@@ -296,42 +351,27 @@ __global__ void __launch_bounds__(512)
   const int64_t c0 = ch * cw;
   const int w = static_cast<int>(kq_min<int64_t>(cw, inner - c0));
   float *g = base + o * so + c0;
-  for (int e = threadIdx.x; e < A * cw; e += blockDim.x) {
-    const int a = e / cw, c = e % cw;
-    X[e] = c < w ? g[a * smid + c] : 0.f;
+  const int R0 = A >= 16 ? 16 : A;
+  const int groups = A / R0;
+  for (int idx = threadIdx.x; idx < groups * cw; idx += blockDim.x) {
+    const int c = idx % cw, gi = idx / cw;
+    float r[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < R0) r[i] = c < w ? g[int64_t(gi * R0 + i) * smid + c] : 0.f;
+    if (R0 == 16) fwht_reg<16>(*reinterpret_cast<float(*)[16]>(r));
+    else if (R0 == 8) fwht_reg<8>(*reinterpret_cast<float(*)[8]>(r));
+    else if (R0 == 4) fwht_reg<4>(*reinterpret_cast<float(*)[4]>(r));
+    else if (R0 == 2) fwht_reg<2>(*reinterpret_cast<float(*)[2]>(r));
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < R0) X[(gi * R0 + i) * cw + c] = r[i];
   }
   __syncthreads();
-  // radix-4 stages, then one radix-2 stage if log2(A) is odd
-  int h = 1;
-  for (; 4 * h <= A; h *= 4) {
-    const int quads = A / 4;
-    for (int idx = threadIdx.x; idx < quads * cw; idx += blockDim.x) {
-      const int c = idx % cw, q = idx / cw;
-      const int a = (q / h) * 4 * h + (q % h);
-      float *x = X + a * cw + c;
-      const float x0 = x[0], x1 = x[h * cw], x2 = x[2 * h * cw], x3 = x[3 * h * cw];
-      const float s0 = x0 + x1, d0 = x0 - x1, s1 = x2 + x3, d1 = x2 - x3;
-      x[0] = s0 + s1;
-      x[h * cw] = d0 + d1;
-      x[2 * h * cw] = s0 - s1;
-      x[3 * h * cw] = d0 - d1;
-    }
-    __syncthreads();
-  }
-  if (h < A) {
-    for (int idx = threadIdx.x; idx < (A / 2) * cw; idx += blockDim.x) {
-      const int c = idx % cw, q = idx / cw;
-      const int a = (q / h) * 2 * h + (q % h);
-      float *x = X + a * cw + c;
-      const float u = x[0], v = x[h * cw];
-      x[0] = u + v;
-      x[h * cw] = u - v;
-    }
-    __syncthreads();
-  }
+  fwht_rest(X, cw, A, R0, cw, [](int v) { return v; });
   for (int e = threadIdx.x; e < A * cw; e += blockDim.x) {
     const int a = e / cw, c = e % cw;
-    if (c < w) g[a * smid + c] = X[e];
+    if (c < w) g[int64_t(a) * smid + c] = X[e];
   }
 }
 
@@ -342,59 +382,27 @@ struct SideRot {
   const float *Q;  // device Q_m (m > 1 and rot) or null
 };
 
-int64_t pow2_floor(int64_t x) {
-  int64_t p = 1;
-  while (p * 2 <= x) p *= 2;
-  return p;
-}
+constexpr int64_t ROW_CHUNK_MAX = 28672;  // floats of one row chunk (112 KB)
+constexpr int SLAB_FLOATS = 32768;        // floats of one strided slab
+constexpr int64_t MAX_A = 1024;           // Hadamard length of one strided pass
 
-kronq_status launch_tile(cudaStream_t st, const TileP &p, int64_t R, int64_t C) {
-  const int TR = p.kr * p.Lr * p.mr, TC = p.kc * p.Lc * p.mc;
-  const int TCP = TC + ((TC & 1) ? 0 : 1);
-  const bool stage = p.Qr || p.Qc;
-  size_t smem = static_cast<size_t>(TR) * TCP * 4 * (stage ? 2 : 1);
-  if (p.Qc && p.mc * p.mc <= 4096) smem += p.mc * p.mc * 4;
-  if (p.Qr && p.mr * p.mr <= 4096) smem += p.mr * p.mr * 4;
-  if (smem > 227 * 1024) return KRONQ_ERR_UNSUPPORTED;
-  if (R % TR || C % TC) return KRONQ_ERR_UNSUPPORTED;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(tile_pass_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             227 * 1024) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr_done = true;
-  }
-  TileP q = p;
-  q.tiles_c = C / TC;
-  const int64_t tiles = (R / TR) * (C / TC);
-  tile_pass_kernel<<<static_cast<unsigned>(tiles), 512, smem, st>>>(q);
-  KQ_CHECK_LAUNCH();
-  return KRONQ_OK;
-}
-
-// Hadamard of length A (power of two) along a strided axis, split into
-// passes of at most MAX_A each (Hhat_A = Hhat_A1 ⊗ Hhat_A2).
 kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
                             int64_t so, int64_t A, int64_t smid, int64_t inner) {
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(strided_fwht_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SLAB_BUDGET * 4) != cudaSuccess)
+                             SLAB_FLOATS * 4) != cudaSuccess)
       return KRONQ_ERR_CUDA;
     attr_done = true;
   }
   int64_t stride = smid;
   while (A > 1) {
     const int64_t a = kq_min<int64_t>(A, MAX_A);
-    // this pass covers the lowest log2(a) bits of the remaining index
-    const int64_t cw = kq_max<int64_t>(1, kq_min<int64_t>(inner, kq_min<int64_t>(256, SLAB_BUDGET / a)));
+    int64_t cw = kq_min<int64_t>(inner, kq_min<int64_t>(256, SLAB_FLOATS / a));
+    cw = kq_max<int64_t>(1, cw);
     const int64_t chunks = ceil_div(inner, cw);
-    // outer index enumerates (outer, high index bits beyond this pass)
     const int64_t hi = A / a;
-    // treat (outer, hi) as one outer axis when they are regularly strided:
-    // element (o, j, t, c) at o*so + (j*a + t)*stride + c for j < hi, t < a
     for (int64_t j = 0; j < hi; ++j) {
       const int64_t blocks = outer * chunks;
       if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
@@ -404,84 +412,89 @@ kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
           static_cast<int>(cw), chunks);
       KQ_CHECK_LAUNCH();
     }
+    // The next pass combines elements `a` positions apart; its independent
+    // vectors are (outer, position within this pass). They form one regular
+    // axis only when the outer axis tiles the current stride exactly.
+    if (A / a > 1) {
+      if (outer * so != stride) return KRONQ_ERR_UNSUPPORTED;
+      outer *= a;
+    }
     stride *= a;
     A /= a;
   }
   return KRONQ_OK;
 }
 
-// out = P_r diag(cr) in diag(cc) P_cᵀ for an R x C matrix (row-major).
+// out = P_r diag(cr) in diag(cc) P_cᵀ for an R x C row-major matrix.
 kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in,
                     float *out, int64_t ld_out, int64_t R, int64_t C,
                     const SideRot &sr, const SideRot &sc, const float *cr,
                     const float *cc) {
   const int64_t had_r = sr.rot ? sr.had : 1, m_r = sr.rot ? sr.m : 1;
   const int64_t had_c = sc.rot ? sc.had : 1, m_c = sc.rot ? sc.m : 1;
-  const bool qr = sr.rot && sr.m > 1, qc = sc.rot && sc.m > 1;
-  const int64_t budget = TILE_BUDGET;
-  // column side block: Lc * m_c, capped at 1024 floats and at the budget / m_r
-  int64_t Lc = 1, Lr = 1, kc = 1, kr = 1;
-  bool split = false;  // Q on both sides does not fit one tile
-  if (qr && qc && m_r * m_c > budget) split = true;
+  // ---- row pass over chunks of Lc * m_c contiguous columns
+  int64_t Lc = 1;
   if (sc.rot) {
-    const int64_t cap = split ? budget / 32 : kq_min<int64_t>(1024, budget / m_r);
-    Lc = pow2_floor(kq_max<int64_t>(1, cap / m_c));
-    while (had_c % Lc) Lc /= 2;
-  }
-  const int64_t tcb = Lc * m_c;
-  if (!sc.rot || tcb < 32) {
-    kc = 1;
-    while (kc * tcb < 32 && C % (2 * kc * tcb) == 0) kc *= 2;
-  }
-  const int64_t TC = kc * tcb;
-  if (!split) {
-    if (sr.rot) {
-      Lr = pow2_floor(kq_max<int64_t>(1, budget / (TC * m_r)));
-      while (had_r % Lr) Lr /= 2;
-      Lr = kq_min<int64_t>(Lr, had_r);
-    }
-    const int64_t trb = Lr * m_r;
-    kr = 1;
-    while (2 * kr * trb * TC <= budget && R % (2 * kr * trb) == 0 && kr * trb < 256)
-      kr *= 2;
-    TileP p{};
-    p.in = in; p.out = out; p.ld_in = ld_in; p.ld_out = ld_out;
-    p.in_bf16 = in_bf16; p.cr = cr; p.cc = cc;
-    p.norm = static_cast<float>(1.0 / sqrt(double(had_r) * double(had_c)));
-    p.kr = kr; p.Lr = Lr; p.mr = m_r; p.kc = kc; p.Lc = Lc; p.mc = m_c;
-    p.Qr = qr ? sr.Q : nullptr;
-    p.Qc = qc ? sc.Q : nullptr;
-    KQ_TRY(launch_tile(st, p, R, C));
+    while (Lc * 2 <= had_c && Lc * 2 * m_c <= ROW_CHUNK_MAX) Lc *= 2;
   } else {
-    // pass 1: column side only (rows independent)
-    TileP p{};
+    // no column rotation: chunks are only a unit of work
+    while (Lc * 2 <= 8192 && C % (Lc * 2) == 0) Lc *= 2;
+  }
+  const int64_t chunk = Lc * m_c;
+  {
+    RowP p{};
     p.in = in; p.out = out; p.ld_in = ld_in; p.ld_out = ld_out;
     p.in_bf16 = in_bf16; p.cr = cr; p.cc = cc;
     p.norm = static_cast<float>(1.0 / sqrt(double(had_r) * double(had_c)));
-    kr = 1;
-    while (2 * kr * TC <= budget && R % (2 * kr) == 0 && kr < 64) kr *= 2;
-    p.kr = kr; p.Lr = 1; p.mr = 1; p.kc = kc; p.Lc = Lc; p.mc = m_c;
-    p.Qc = sc.Q;
-    KQ_TRY(launch_tile(st, p, R, C));
-    // pass 2: row side only (columns independent), in place on out
-    TileP q{};
-    q.in = out; q.out = out; q.ld_in = ld_out; q.ld_out = ld_out;
-    q.in_bf16 = 0; q.norm = 1.f;
-    Lr = pow2_floor(kq_max<int64_t>(1, budget / (32 * m_r)));
-    while (had_r % Lr) Lr /= 2;
-    int64_t kc2 = 1;
-    while (Lr * m_r * 2 * kc2 <= budget && C % (2 * kc2) == 0 && kc2 < 32) kc2 *= 2;
-    q.kr = 1; q.Lr = Lr; q.mr = m_r; q.kc = kc2; q.Lc = 1; q.mc = 1;
-    q.Qr = sr.Q;
-    KQ_TRY(launch_tile(st, q, R, C));
+    p.L = static_cast<int>(sc.rot ? Lc : chunk);
+    p.m = static_cast<int>(sc.rot ? m_c : 1);
+    if (!sc.rot) p.L = static_cast<int>(chunk), p.m = 1;
+    p.Q = (sc.rot && m_c > 1) ? sc.Q : nullptr;
+    p.chunks = C / chunk;
+    size_t smem = static_cast<size_t>(chunk) * 4;
+    static bool attr_done = false;
+    if (!attr_done) {
+      if (cudaFuncSetAttribute(row_pass_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ROW_CHUNK_MAX * 4) != cudaSuccess)
+        return KRONQ_ERR_CUDA;
+      attr_done = true;
+    }
+    if (C % chunk) return KRONQ_ERR_UNSUPPORTED;
+    const int64_t blocks = R * p.chunks;
+    if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+    // without a column rotation the chunk is a plain scaled copy: L = chunk
+    // with no Hadamard would be wrong, so run it as m = chunk, L = 1
+    if (!sc.rot) {
+      p.L = 1;
+      p.m = static_cast<int>(chunk);
+      p.Q = nullptr;
+    }
+    row_pass_kernel<<<static_cast<unsigned>(blocks), 512, smem, st>>>(p);
+    KQ_CHECK_LAUNCH();
   }
-  // remaining Hadamard bits
-  const int64_t Ac = had_c / Lc, Ar = had_r / Lr;
-  if (Ac > 1) KQ_TRY(launch_strided(st, out, R, ld_out, Ac, tcb, tcb));
-  if (Ar > 1) {
-    const int64_t blk = Lr * m_r;  // rows per block
-    KQ_TRY(launch_strided(st, out, blk, ld_out, Ar, blk * ld_out, C));
+  // ---- column-side Hadamard bits beyond the chunk
+  if (sc.rot && had_c / Lc > 1)
+    KQ_TRY(launch_strided(st, out, R, ld_out, had_c / Lc, chunk, chunk));
+  // ---- row side: Q_m over groups of m_r consecutive rows, then the Hadamard
+  if (sr.rot && m_r > 1) {
+    const size_t smem = (static_cast<size_t>(m_r) * m_r + (m_r > 32 ? m_r * 64 : 0)) * 4;
+    if (smem > 227 * 1024) return KRONQ_ERR_UNSUPPORTED;
+    static bool attr_done = false;
+    if (!attr_done) {
+      if (cudaFuncSetAttribute(rowq_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) != cudaSuccess)
+        return KRONQ_ERR_CUDA;
+      attr_done = true;
+    }
+    const int64_t cols = m_r > 32 ? 64 : 256;
+    dim3 grid(static_cast<unsigned>(ceil_div(C, cols)), static_cast<unsigned>(had_r));
+    rowq_kernel<<<grid, 256, smem, st>>>(out, ld_out, C, static_cast<int>(m_r), sr.Q);
+    KQ_CHECK_LAUNCH();
   }
+  if (sr.rot && had_r > 1)
+    KQ_TRY(launch_strided(st, out, m_r, ld_out, had_r, m_r * ld_out, C));
   return KRONQ_OK;
 }
 

@@ -6,8 +6,9 @@
 // layer loss. One CTA computes a 128x128 tile:
 //   warp 0      TMA producer (one elected lane), 3-stage ring of 32-wide k-slabs
 //   warp 1      TMEM owner and MMA issuer (one elected lane)
-//   warps 2..5  split each landed fp32 slab into hi/lo in shared memory, then
-//               run the epilogue (TMEM -> registers -> C).
+//   warps 2..5  write the TF32 low part of each landed fp32 slab next to it in
+//               shared memory (the raw slab itself serves as the high part),
+//               then run the epilogue (TMEM -> registers -> C).
 #include "kernels.cuh"
 
 namespace kronq {
@@ -30,15 +31,15 @@ struct Ctl {
 };
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + sizeof(Ctl) + 64;
 
-__device__ __forceinline__ void split_tf32(float4 &hi, float4 &lo) {
+// The tf32 MMA reads an fp32 operand by dropping its 13 low mantissa bits
+// (truncation, measured on sm_100a), so the raw slab already is the hi part;
+// only lo = x - trunc(x) (exact in fp32) has to be written.
+__device__ __forceinline__ float4 tf32_lo(float4 x) {
   const uint32_t mask = 0xffffe000u;
-  float4 h;
-  h.x = __uint_as_float(__float_as_uint(hi.x) & mask);
-  h.y = __uint_as_float(__float_as_uint(hi.y) & mask);
-  h.z = __uint_as_float(__float_as_uint(hi.z) & mask);
-  h.w = __uint_as_float(__float_as_uint(hi.w) & mask);
-  lo = make_float4(hi.x - h.x, hi.y - h.y, hi.z - h.z, hi.w - h.w);
-  hi = h;
+  return make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & mask),
+                     x.y - __uint_as_float(__float_as_uint(x.y) & mask),
+                     x.z - __uint_as_float(__float_as_uint(x.z) & mask),
+                     x.w - __uint_as_float(__float_as_uint(x.w) & mask));
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -182,14 +183,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr int Q = TILE_BYTES / 16;
 #pragma unroll 4
       for (int i = ct; i < Q; i += 128) {
-        float4 a = st[i], al;
-        split_tf32(a, al);
-        st[i] = a;
-        st[Q + i] = al;
-        float4 b = st[2 * Q + i], bl;
-        split_tf32(b, bl);
-        st[2 * Q + i] = b;
-        st[3 * Q + i] = bl;
+        st[Q + i] = tf32_lo(st[i]);
+        st[3 * Q + i] = tf32_lo(st[2 * Q + i]);
       }
       fence_proxy_async_smem();
       mbar_arrive(&ctl->conv[s]);

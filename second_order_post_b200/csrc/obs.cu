@@ -19,15 +19,19 @@ namespace kronq {
 namespace {
 
 constexpr int OB = 128;        // block width
-constexpr int OTHREADS = 512;  // 16 warps
-constexpr int ROWS_PER_WARP = 4;
-constexpr int OROWS = (OTHREADS / 32) * ROWS_PER_WARP;
+constexpr int OTHREADS = 256;  // 8 warps
+constexpr int RPW = 4;         // rows per warp, swept together
+constexpr int OROWS = (OTHREADS / 32) * RPW;
 constexpr int SUPER = 1024;    // super-block width
+constexpr int OSMEM = (OB * OB + OB) * 4;
 
 __device__ __forceinline__ float pick4(const float (&v)[4], int s) {
   return s == 0 ? v[0] : s == 1 ? v[1] : s == 2 ? v[2] : v[3];
 }
 
+// One 128-column block for OROWS rows per CTA. Each warp sweeps its 4 rows
+// together (independent dependency chains), lane l holding columns
+// l, l+32, l+64, l+96 of each row.
 __global__ void __launch_bounds__(OTHREADS)
     obs_block_kernel(float *__restrict__ W, int64_t ldw,
                      const float *__restrict__ U, int64_t ldu, int64_t j0,
@@ -36,95 +40,116 @@ __global__ void __launch_bounds__(OTHREADS)
                      uint32_t *__restrict__ codes, int64_t ldq,
                      float *__restrict__ scales, uint8_t *__restrict__ zeros,
                      int64_t ngroups) {
-  extern __shared__ float Us[];                      // OB x OB
-  __shared__ uint8_t qsm[OTHREADS / 32][OB];
+  extern __shared__ float Us[];                 // OB x OB, then 1/U[j][j]
+  float *inv = Us + OB * OB;
+  __shared__ uint8_t qsm[OTHREADS / 32][RPW][OB];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < OB * OB; e += OTHREADS) {
     const int r = e / OB, c = e % OB;
     Us[e] = U[(j0 + r) * ldu + j0 + c];
   }
   __syncthreads();
+  if (threadIdx.x < OB) inv[threadIdx.x] = 1.f / Us[threadIdx.x * OB + threadIdx.x];
+  __syncthreads();
   const float maxq = static_cast<float>((1 << bits) - 1);
-  for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
-    const int64_t row =
-        int64_t(blockIdx.x) * OROWS + warp * ROWS_PER_WARP + rr;
-    if (row >= d_out) break;
-    float w[4], err[4], qv[4];
-    float *wrow = W + row * ldw + j0;
+  const int64_t row0 = int64_t(blockIdx.x) * OROWS + warp * RPW;
+  float w[RPW][4], err[RPW][4];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    const bool ok = row0 + r < d_out;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      w[s] = wrow[lane + 32 * s];
-      err[s] = 0.f;
-      qv[s] = 0.f;
+      w[r][s] = ok ? W[(row0 + r) * ldw + j0 + lane + 32 * s] : 0.f;
+      err[r][s] = 0.f;
     }
-    float scale = 1.f, zero = 0.f;
-    for (int j = 0; j < OB; ++j) {
-      if (j % group == 0) {
-        float mn = INFINITY, mx = -INFINITY;
+  }
+  float scale[RPW], zero[RPW];
+  for (int j = 0; j < OB; ++j) {
+    if (j % group == 0) {
+      float mn[RPW], mx[RPW];
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        mn[r] = INFINITY;
+        mx[r] = -INFINITY;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const int c = lane + 32 * s;
           if (c >= j && c < j + group) {
-            mn = fminf(mn, w[s]);
-            mx = fmaxf(mx, w[s]);
+            mn[r] = fminf(mn[r], w[r][s]);
+            mx[r] = fmaxf(mx[r], w[r][s]);
           }
         }
+      }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
         }
-        const float xmin = fminf(mn, 0.f), xmax = fmaxf(mx, 0.f);
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        const float xmin = fminf(mn[r], 0.f), xmax = fmaxf(mx[r], 0.f);
         if (xmax == xmin) {
-          scale = 1.f;
-          zero = 0.f;
+          scale[r] = 1.f;
+          zero[r] = 0.f;
         } else {
-          scale = (xmax - xmin) / maxq;
-          zero = rintf(-xmin / scale);
+          scale[r] = (xmax - xmin) / maxq;
+          zero[r] = rintf(-xmin / scale[r]);
         }
-        if (lane == 0) {
+        if (lane == 0 && row0 + r < d_out) {
           const int64_t gi = (j0 + j) / group;
-          scales[row * ngroups + gi] = scale;
-          zeros[row * ngroups + gi] = static_cast<uint8_t>(zero);
+          scales[(row0 + r) * ngroups + gi] = scale[r];
+          zeros[(row0 + r) * ngroups + gi] = static_cast<uint8_t>(zero[r]);
         }
       }
-      const int slot = j >> 5, owner = j & 31;
-      const float wj = __shfl_sync(0xffffffffu, pick4(w, slot), owner);
-      const float q = fminf(fmaxf(rintf(wj / scale) + zero, 0.f), maxq);
-      const float wh = scale * (q - zero);
-      const float e = (wj - wh) / Us[j * OB + j];
-      const float *urow = Us + j * OB;
+    }
+    const int slot = j >> 5, owner = j & 31;
+    const float *urow = Us + j * OB;
+    float u[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) u[s] = urow[lane + 32 * s];
+    const float iu = inv[j];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float wj = __shfl_sync(0xffffffffu, pick4(w[r], slot), owner);
+      const float q = fminf(fmaxf(rintf(wj / scale[r]) + zero[r], 0.f), maxq);
+      const float wh = scale[r] * (q - zero[r]);
+      const float e = (wj - wh) * iu;
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const int c = lane + 32 * s;
-        if (c > j) w[s] = fmaf(-e, urow[c], w[s]);
+        if (c > j) w[r][s] = fmaf(-e, u[s], w[r][s]);
         if (s == slot && lane == owner) {
-          w[s] = wh;
-          err[s] = e;
-          qv[s] = q;
+          w[r][s] = wh;
+          err[r][s] = e;
         }
       }
+      if (lane == owner) qsm[warp][r][j] = static_cast<uint8_t>(q);
     }
+  }
+  __syncwarp();
+  const int nwords = OB * bits / 32;
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    const int64_t row = row0 + r;
+    if (row >= d_out) break;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      wrow[lane + 32 * s] = w[s];
-      E[row * lde + e_col + lane + 32 * s] = err[s];
-      qsm[warp][lane + 32 * s] = static_cast<uint8_t>(qv[s]);
+      W[row * ldw + j0 + lane + 32 * s] = w[r][s];
+      E[row * lde + e_col + lane + 32 * s] = err[r][s];
     }
-    __syncwarp();
-    const int nwords = OB * bits / 32;
     if (lane < nwords) {
       uint32_t word = 0;
       const int bit0 = 32 * lane;
       const int c_lo = bit0 / bits, c_hi = min(OB - 1, (bit0 + 31) / bits);
       for (int c = c_lo; c <= c_hi; ++c) {
         const int sh = c * bits - bit0;
-        const uint32_t code = qsm[warp][c];
+        const uint32_t code = qsm[warp][r][c];
         word |= sh >= 0 ? (code << sh) : (code >> (-sh));
       }
       codes[row * ldq + (j0 * bits) / 32 + lane] = word;
     }
-    __syncwarp();
   }
 }
 
@@ -148,7 +173,7 @@ kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
   if (!attr_done) {
     if (cudaFuncSetAttribute(obs_block_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             OB * OB * 4) != cudaSuccess)
+                             OSMEM) != cudaSuccess)
       return KRONQ_ERR_CUDA;
     attr_done = true;
   }
@@ -156,7 +181,7 @@ kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
   for (int64_t sb0 = 0; sb0 < d_in; sb0 += S) {
     const int64_t sb1 = kq_min<int64_t>(d_in, sb0 + S);
     for (int64_t j0 = sb0; j0 < sb1; j0 += OB) {
-      obs_block_kernel<<<grid, OTHREADS, OB * OB * 4, st>>>(
+      obs_block_kernel<<<grid, OTHREADS, OSMEM, st>>>(
           W, d_in, U, d_in, j0, d_out, o.bits, o.group, E, S, j0 - sb0, codes,
           ldq, scales, zeros, ngroups);
       KQ_CHECK_LAUNCH();
