@@ -7,12 +7,14 @@
 //
 // Every rotation of an R x C row-major matrix M -> P_r diag(cr) M diag(cc) P_cᵀ
 // is split into memory passes whose working sets fit in shared memory:
-//   tile pass     one (kr*Lr*mr) x (kc*Lc*mc) tile per CTA: input factors,
-//                 Hadamard over the low Lc (Lr) index bits and Q_m on the
-//                 contiguous (consecutive-row) factor of each side
-//   strided pass  Hadamard over the remaining high index bits, whose elements
-//                 sit at a fixed stride (within a row, or across rows); one
-//                 [A][cw] slab per CTA with cw contiguous columns
+//   row pass      one row chunk of Lc*m_c contiguous columns per CTA: input
+//                 factors, Hadamard over the chunk's a-index, Q_m over each
+//                 group of m_c contiguous values (the whole column side when
+//                 the row fits in 112 KB)
+//   row-side Q_m  groups of m_r consecutive rows, one thread per column
+//   strided pass  Hadamard over index bits whose elements sit at a fixed
+//                 stride (within a row, or across rows); one [A][cw] slab per
+//                 CTA with cw contiguous columns
 // The Hadamard factors commute with each other and with Q_m (Kronecker
 // structure), so the order of the passes does not change the result.
 #include <math.h>
@@ -238,7 +240,7 @@ __device__ void row_load_round(const RowP &p, float *X, int64_t row, int64_t c0)
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(512) row_pass_kernel(RowP p) {
+__global__ void __launch_bounds__(512, 2) row_pass_kernel(RowP p) {
   extern __shared__ float X[];
   const int m = p.m, L = p.L, chunk = L * m;
   const int64_t row = blockIdx.x / p.chunks;
@@ -268,8 +270,37 @@ __global__ void __launch_bounds__(512) row_pass_kernel(RowP p) {
     return;
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  if (m <= 32) {
-    // lane b owns output b of every group; its row of Q_m stays in registers
+  if (m <= 32 && (m % 4) == 0) {
+    // lane b owns output b of every group; its row of Q_m stays in registers;
+    // two groups per iteration, inputs read as float4 broadcasts
+    float q[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) q[k] = (lane < m && k < m) ? p.Q[lane * m + k] : 0.f;
+    for (int a = 2 * warp; a < L; a += 2 * nw) {
+      const bool two = a + 1 < L;
+      const float4 *x0 = reinterpret_cast<const float4 *>(X + a * m);
+      const float4 *x1 = reinterpret_cast<const float4 *>(X + (two ? a + 1 : a) * m);
+      float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        if (4 * k4 < m) {
+          const float4 u = x0[k4], v = x1[k4];
+          y0 = fmaf(q[4 * k4], u.x, y0);
+          y0 = fmaf(q[4 * k4 + 1], u.y, y0);
+          y0 = fmaf(q[4 * k4 + 2], u.z, y0);
+          y0 = fmaf(q[4 * k4 + 3], u.w, y0);
+          y1 = fmaf(q[4 * k4], v.x, y1);
+          y1 = fmaf(q[4 * k4 + 1], v.y, y1);
+          y1 = fmaf(q[4 * k4 + 2], v.z, y1);
+          y1 = fmaf(q[4 * k4 + 3], v.w, y1);
+        }
+      }
+      if (lane < m) {
+        o[a * m + lane] = y0;
+        if (two) o[(a + 1) * m + lane] = y1;
+      }
+    }
+  } else if (m <= 32) {
     float q[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) q[k] = (lane < m && k < m) ? p.Q[lane * m + k] : 0.f;
@@ -301,7 +332,10 @@ __global__ void __launch_bounds__(512) row_pass_kernel(RowP p) {
 __global__ void __launch_bounds__(256)
     rowq_kernel(float *M, int64_t ld, int64_t C, int m, const float *Q) {
   extern __shared__ float sm[];  // Q (m*m), then a [m][64] tile when m > 32
-  for (int e = threadIdx.x; e < m * m; e += blockDim.x) sm[e] = Q[e];
+  for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
+    sm[e] = Q[e];
+    if (m <= 32) sm[m * m + (e % m) * m + e / m] = Q[e];  // Qᵀ
+  }
   __syncthreads();
   const int64_t a = blockIdx.y;
   float *base = M + a * m * ld;
@@ -311,13 +345,35 @@ __global__ void __launch_bounds__(256)
     float x[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) x[k] = k < m ? base[k * ld + c] : 0.f;
-    for (int b = 0; b < m; ++b) {
-      const float *qr = sm + b * m;
-      float y = 0.f;
+    if (m % 4 == 0) {
+      // Qᵀ (k-major) in shared memory: 4 outputs per float4 broadcast
+      const float4 *qt = reinterpret_cast<const float4 *>(sm + m * m);
+      for (int b0 = 0; b0 < m; b0 += 4) {
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        if (k < m) y = fmaf(qr[k], x[k], y);
-      base[b * ld + c] = y;
+        for (int k = 0; k < 32; ++k) {
+          if (k < m) {
+            const float4 qv = qt[(k * m + b0) / 4];
+            y0 = fmaf(qv.x, x[k], y0);
+            y1 = fmaf(qv.y, x[k], y1);
+            y2 = fmaf(qv.z, x[k], y2);
+            y3 = fmaf(qv.w, x[k], y3);
+          }
+        }
+        base[b0 * ld + c] = y0;
+        base[(b0 + 1) * ld + c] = y1;
+        base[(b0 + 2) * ld + c] = y2;
+        base[(b0 + 3) * ld + c] = y3;
+      }
+    } else {
+      for (int b = 0; b < m; ++b) {
+        const float *qr = sm + b * m;
+        float y = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (k < m) y = fmaf(qr[k], x[k], y);
+        base[b * ld + c] = y;
+      }
     }
   } else {
     float *T = sm + m * m;  // [m][64]
@@ -340,6 +396,107 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------- strided pass
+// Vector form: cw contiguous columns as float4 lanes; the first Hadamard round
+// runs in registers while loading, the last one while storing, and only the
+// rounds in between touch shared memory. Needs 16-byte aligned rows.
+template <int R>
+__device__ __forceinline__ void fwht_reg4(float4 (&r)[R]) {
+#pragma unroll
+  for (int s = 1; s < R; s <<= 1)
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      if (!(i & s)) {
+        const float4 u = r[i], w = r[i + s];
+        r[i] = make_float4(u.x + w.x, u.y + w.y, u.z + w.z, u.w + w.w);
+        r[i + s] = make_float4(u.x - w.x, u.y - w.y, u.z - w.z, u.w - w.w);
+      }
+}
+
+template <int R>
+__device__ void round4_load(float4 *X, const float4 *g, int A, int c4n, int64_t smid4,
+                            int w4) {
+  const int groups = A / R;
+  for (int idx = threadIdx.x; idx < groups * c4n; idx += blockDim.x) {
+    const int c = idx % c4n, gi = idx / c4n;
+    float4 r[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      r[i] = c < w4 ? g[int64_t(gi * R + i) * smid4 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    fwht_reg4<R>(r);
+#pragma unroll
+    for (int i = 0; i < R; ++i) X[(gi * R + i) * c4n + c] = r[i];
+  }
+  __syncthreads();
+}
+
+template <int R>
+__device__ void round4_smem(float4 *X, int A, int h, int c4n) {
+  const int groups = A / R;
+  for (int idx = threadIdx.x; idx < groups * c4n; idx += blockDim.x) {
+    const int c = idx % c4n, g = idx / c4n;
+    const int a = (g / h) * R * h + (g % h);
+    float4 r[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) r[i] = X[(a + i * h) * c4n + c];
+    fwht_reg4<R>(r);
+#pragma unroll
+    for (int i = 0; i < R; ++i) X[(a + i * h) * c4n + c] = r[i];
+  }
+  __syncthreads();
+}
+
+template <int R>
+__device__ void round4_store(const float4 *X, float4 *g, int A, int h, int c4n,
+                             int64_t smid4, int w4) {
+  const int groups = A / R;
+  for (int idx = threadIdx.x; idx < groups * c4n; idx += blockDim.x) {
+    const int c = idx % c4n, gg = idx / c4n;
+    const int a = (gg / h) * R * h + (gg % h);
+    float4 r[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) r[i] = X[(a + i * h) * c4n + c];
+    fwht_reg4<R>(r);
+    if (c < w4) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) g[int64_t(a + i * h) * smid4 + c] = r[i];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(512)
+    strided_fwht4_kernel(float *base, int64_t so, int A, int64_t smid,
+                         int64_t inner, int cw, int64_t chunks) {
+  extern __shared__ float4 X4[];
+  const int64_t o = blockIdx.x / chunks, ch = blockIdx.x % chunks;
+  const int64_t c0 = ch * cw;
+  const int w4 = static_cast<int>(kq_min<int64_t>(cw, inner - c0)) / 4;
+  float4 *g = reinterpret_cast<float4 *>(base + o * so + c0);
+  const int c4n = cw / 4;
+  const int64_t smid4 = smid / 4;
+  const int R0 = A >= 16 ? 16 : A;
+  switch (R0) {
+    case 16: round4_load<16>(X4, g, A, c4n, smid4, w4); break;
+    case 8: round4_load<8>(X4, g, A, c4n, smid4, w4); break;
+    case 4: round4_load<4>(X4, g, A, c4n, smid4, w4); break;
+    case 2: round4_load<2>(X4, g, A, c4n, smid4, w4); break;
+    default: round4_load<1>(X4, g, A, c4n, smid4, w4); break;
+  }
+  int h = R0;
+  while (A / h > 16) {
+    round4_smem<16>(X4, A, h, c4n);
+    h *= 16;
+  }
+  switch (A / h) {
+    case 16: round4_store<16>(X4, g, A, h, c4n, smid4, w4); break;
+    case 8: round4_store<8>(X4, g, A, h, c4n, smid4, w4); break;
+    case 4: round4_store<4>(X4, g, A, h, c4n, smid4, w4); break;
+    case 2: round4_store<2>(X4, g, A, h, c4n, smid4, w4); break;
+    default: round4_store<1>(X4, g, A, h, c4n, smid4, w4); break;
+  }
+}
+
+// Scalar form of the strided pass (any alignment).
+
 // View [outer][A][inner] at strides (so, smid, 1); Hadamard (unnormalised) of
 // length A along the middle axis; one [A][cw] slab per CTA, first radix-16
 // round in registers while loading.
@@ -392,10 +549,15 @@ kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
   if (!attr_done) {
     if (cudaFuncSetAttribute(strided_fwht_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SLAB_FLOATS * 4) != cudaSuccess ||
+        cudaFuncSetAttribute(strided_fwht4_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SLAB_FLOATS * 4) != cudaSuccess)
       return KRONQ_ERR_CUDA;
     attr_done = true;
   }
+  const bool vec = reinterpret_cast<uintptr_t>(base) % 16 == 0 && so % 4 == 0 &&
+                   smid % 4 == 0 && inner % 4 == 0;
   int64_t stride = smid;
   while (A > 1) {
     const int64_t a = kq_min<int64_t>(A, MAX_A);
@@ -406,10 +568,16 @@ kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
     for (int64_t j = 0; j < hi; ++j) {
       const int64_t blocks = outer * chunks;
       if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
-      strided_fwht_kernel<<<static_cast<unsigned>(blocks), 512,
-                            static_cast<size_t>(a * cw * 4), st>>>(
-          base + j * a * stride, so, static_cast<int>(a), stride, inner,
-          static_cast<int>(cw), chunks);
+      if (vec && cw % 4 == 0)
+        strided_fwht4_kernel<<<static_cast<unsigned>(blocks), 512,
+                               static_cast<size_t>(a * cw * 4), st>>>(
+            base + j * a * stride, so, static_cast<int>(a), stride, inner,
+            static_cast<int>(cw), chunks);
+      else
+        strided_fwht_kernel<<<static_cast<unsigned>(blocks), 512,
+                              static_cast<size_t>(a * cw * 4), st>>>(
+            base + j * a * stride, so, static_cast<int>(a), stride, inner,
+            static_cast<int>(cw), chunks);
       KQ_CHECK_LAUNCH();
     }
     // The next pass combines elements `a` positions apart; its independent
@@ -478,7 +646,9 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
     KQ_TRY(launch_strided(st, out, R, ld_out, had_c / Lc, chunk, chunk));
   // ---- row side: Q_m over groups of m_r consecutive rows, then the Hadamard
   if (sr.rot && m_r > 1) {
-    const size_t smem = (static_cast<size_t>(m_r) * m_r + (m_r > 32 ? m_r * 64 : 0)) * 4;
+    // Q_m, then Qᵀ (m <= 32) or a [m][64] input tile (m > 32)
+    const size_t smem =
+        (static_cast<size_t>(m_r) * m_r + (m_r > 32 ? m_r * 64 : m_r * m_r)) * 4;
     if (smem > 227 * 1024) return KRONQ_ERR_UNSUPPORTED;
     static bool attr_done = false;
     if (!attr_done) {

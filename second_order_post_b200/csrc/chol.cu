@@ -43,65 +43,89 @@ __global__ void damping_kernel(const float *H, int64_t d, float damp_rel,
   }
 }
 
+// Sweep-1 step for one row: row[k] -= colj[k*LP] * f for k = k0, k0+4, ... < j.
+// The row (A[i][k], k < j) and the pivot column (A[k][j]) never share an
+// element, so the loads can run ahead of the stores.
+__device__ __forceinline__ void ldl_row_step(float *__restrict__ row,
+                                             const float *__restrict__ colj,
+                                             int k0, int j, float f) {
+#pragma unroll 4
+  for (int k = k0; k < j; k += 4) row[k] = fmaf(-colj[k * LP], f, row[k]);
+}
+
 // One diagonal leaf at rows/cols [off, off+NB): reads the upper triangle of the
 // (already updated) block, adds λ, writes U (upper, zeros below).
+// Sweep 1, reverse LDLᵀ in shared memory: thread (row i, residue q) updates
+// A[i][k] for k ≡ q (mod 4); warps are numbered so that each scheduler holds
+// all four row blocks of one residue (balanced). One barrier per column.
+// Sweep 2, X = (unit upper)^-1 one column at a time from the bottom row up:
+// four lanes of a warp share a column and split the k-sum, no block barrier.
 __global__ void __launch_bounds__(LTHREADS)
     chol_leaf_kernel(float *__restrict__ H, int64_t ld, int64_t off,
                      const float *__restrict__ lambda, int32_t *info) {
   extern __shared__ float sm[];
-  float *A = sm;              // NB x LP: pivots / LDLᵀ factor
-  float *X = sm + NB * LP;    // NB x LP: inverse of the unit triangle
-  __shared__ int bad;
-  const int t = threadIdx.x;
-  const int col = t % NB;     // column owned by this thread
-  const int r0 = t / NB;      // rows r0, r0+4, ...
+  float *A = sm;                 // NB x LP
+  float *X = sm + NB * LP;       // NB x LP
+  float *piv = X + NB * LP;      // NB pivots
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const float lam = *lambda;
-  if (t == 0) bad = 0;
   for (int e = t; e < NB * NB; e += LTHREADS) {
     const int r = e / NB, c = e % NB;
     if (c >= r) {
       float v = H[(off + r) * ld + off + c];
       if (c == r) v += lam;
       A[r * LP + c] = v;
-      A[c * LP + r] = v;
     }
   }
   __syncthreads();
-  // reverse LDLᵀ: for j = NB-1..0, A[i][k] -= A[i][j] A[k][j] / A[j][j], i<=k<j
-  for (int j = NB - 1; j >= 0; --j) {
-    const float piv = A[j * LP + j];
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      if (t == 0 && !bad) {
-        bad = 1;
-        report(info, KRONQ_ERR_NOT_PD | static_cast<int32_t>((off + j) << 8));
+  // ---- sweep 1
+  {
+    const int q = w & 3, i = 32 * (w >> 2) + lane;
+    const int k0 = i + ((q - i) & 3);  // first k >= i with k ≡ q (mod 4)
+    bool bad = false;
+    for (int j = NB - 1; j >= 0; --j) {
+      const float p = A[j * LP + j];
+      if (t == 0) {
+        piv[j] = p;
+        if (!(p > 0.f) || !isfinite(p)) {
+          if (!bad) report(info, KRONQ_ERR_NOT_PD | static_cast<int32_t>((off + j) << 8));
+          bad = true;
+        }
       }
+      if (i < j) ldl_row_step(A + i * LP, A + j, k0, j, A[i * LP + j] / p);
+      __syncthreads();
     }
-    if (col < j) {
-      const float f = A[col * LP + j] / piv;
-      for (int i = r0; i <= col; i += 4) A[i * LP + col] -= A[i * LP + j] * f;
-    }
-    __syncthreads();
   }
-  // unit upper factor (in place above the diagonal) and X = I
+  // unit upper factor in place: A[i][k] / piv[k], i < k
   for (int e = t; e < NB * NB; e += LTHREADS) {
     const int r = e / NB, c = e % NB;
-    if (c > r) A[r * LP + c] /= A[c * LP + c];
-    X[r * LP + c] = (r == c) ? 1.f : 0.f;
+    if (c > r) A[r * LP + c] /= piv[c];
   }
   __syncthreads();
-  // X = (unit upper)^-1: for k = NB-1..1, X[i][c] -= A[i][k] X[k][c], i<k<=c
-  for (int k = NB - 1; k >= 1; --k) {
-    if (col >= k) {
-      const float xk = X[k * LP + col];
-      for (int i = r0; i < k; i += 4) X[i * LP + col] -= A[i * LP + k] * xk;
+  // ---- sweep 2: column c of X, lanes 4g..4g+3 of a warp share c
+  {
+    const int part = lane & 3;
+    const int c = 8 * w + (lane >> 2);
+    X[c * LP + c] = 1.f;  // X stored transposed: X[c][i] holds X(i, c)
+    __syncwarp();
+    float *xc = X + c * LP;
+    for (int i = NB - 2; i >= 0; --i) {
+      float s = 0.f;
+      if (i < c) {
+        const float *ri = A + i * LP;
+        for (int k = i + 1 + part; k <= c; k += 4) s = fmaf(ri[k], xc[k], s);
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (part == 0 && i < c) xc[i] = -s;
+      __syncwarp();
     }
-    __syncthreads();
   }
-  // U = D^-1/2 X
+  __syncthreads();
+  // U(i, c) = X(i, c) / sqrt(piv[i]) for i <= c, zeros below the diagonal
   for (int e = t; e < NB * NB; e += LTHREADS) {
-    const int r = e / NB, c = e % NB;
-    const float piv = A[r * LP + r];
-    H[(off + r) * ld + off + c] = (c >= r) ? X[r * LP + c] / sqrtf(piv) : 0.f;
+    const int i = e / NB, c = e % NB;
+    H[(off + i) * ld + off + c] = (i <= c) ? X[c * LP + i] / sqrtf(piv[i]) : 0.f;
   }
 }
 
@@ -126,7 +150,7 @@ struct Ctx {
 inline int64_t first_half(int64_t n) { return (n / NB / 2) * NB; }
 
 kronq_status leaf(const Ctx &c, int64_t off) {
-  const int smem = 2 * NB * LP * sizeof(float);
+  const int smem = (2 * NB * LP + NB) * sizeof(float);
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(chol_leaf_kernel,
