@@ -464,13 +464,13 @@ __device__ void round4_store(const float4 *X, float4 *g, int A, int h, int c4n,
 }
 
 __global__ void __launch_bounds__(512)
-    strided_fwht4_kernel(float *base, int64_t so, int A, int64_t smid,
-                         int64_t inner, int cw, int64_t chunks) {
+    strided_fwht4_kernel(float *base, int64_t so, int64_t n1, int64_t so2, int A,
+                         int64_t smid, int64_t inner, int cw, int64_t chunks) {
   extern __shared__ float4 X4[];
   const int64_t o = blockIdx.x / chunks, ch = blockIdx.x % chunks;
   const int64_t c0 = ch * cw;
   const int w4 = static_cast<int>(kq_min<int64_t>(cw, inner - c0)) / 4;
-  float4 *g = reinterpret_cast<float4 *>(base + o * so + c0);
+  float4 *g = reinterpret_cast<float4 *>(base + (o % n1) * so + (o / n1) * so2 + c0);
   const int c4n = cw / 4;
   const int64_t smid4 = smid / 4;
   const int R0 = A >= 16 ? 16 : A;
@@ -501,13 +501,13 @@ __global__ void __launch_bounds__(512)
 // length A along the middle axis; one [A][cw] slab per CTA, first radix-16
 // round in registers while loading.
 __global__ void __launch_bounds__(512)
-    strided_fwht_kernel(float *base, int64_t so, int A, int64_t smid,
-                        int64_t inner, int cw, int64_t chunks) {
+    strided_fwht_kernel(float *base, int64_t so, int64_t n1, int64_t so2, int A,
+                        int64_t smid, int64_t inner, int cw, int64_t chunks) {
   extern __shared__ float X[];
   const int64_t o = blockIdx.x / chunks, ch = blockIdx.x % chunks;
   const int64_t c0 = ch * cw;
   const int w = static_cast<int>(kq_min<int64_t>(cw, inner - c0));
-  float *g = base + o * so + c0;
+  float *g = base + (o % n1) * so + (o / n1) * so2 + c0;
   const int R0 = A >= 16 ? 16 : A;
   const int groups = A / R0;
   for (int idx = threadIdx.x; idx < groups * cw; idx += blockDim.x) {
@@ -543,6 +543,10 @@ constexpr int64_t ROW_CHUNK_MAX = 28672;  // floats of one row chunk (112 KB)
 constexpr int SLAB_FLOATS = 32768;        // floats of one strided slab
 constexpr int64_t MAX_A = 1024;           // Hadamard length of one strided pass
 
+// Hadamard of length A (power of two) along the middle axis of the view
+// [outer][A][inner] (strides so, smid, 1). Lengths above MAX_A are split into
+// two balanced factors Hhat_A = Hhat_hi ⊗ Hhat_lo, one pass each; each pass
+// sees its independent vectors on a two-level outer index.
 kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
                             int64_t so, int64_t A, int64_t smid, int64_t inner) {
   static bool attr_done = false;
@@ -556,41 +560,37 @@ kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
       return KRONQ_ERR_CUDA;
     attr_done = true;
   }
+  if (A <= 1) return KRONQ_OK;
   const bool vec = reinterpret_cast<uintptr_t>(base) % 16 == 0 && so % 4 == 0 &&
                    smid % 4 == 0 && inner % 4 == 0;
-  int64_t stride = smid;
-  while (A > 1) {
-    const int64_t a = kq_min<int64_t>(A, MAX_A);
+  auto pass = [&](int64_t a, int64_t stride, int64_t n2, int64_t so2) -> kronq_status {
     int64_t cw = kq_min<int64_t>(inner, kq_min<int64_t>(256, SLAB_FLOATS / a));
     cw = kq_max<int64_t>(1, cw);
     const int64_t chunks = ceil_div(inner, cw);
-    const int64_t hi = A / a;
-    for (int64_t j = 0; j < hi; ++j) {
-      const int64_t blocks = outer * chunks;
-      if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
-      if (vec && cw % 4 == 0)
-        strided_fwht4_kernel<<<static_cast<unsigned>(blocks), 512,
-                               static_cast<size_t>(a * cw * 4), st>>>(
-            base + j * a * stride, so, static_cast<int>(a), stride, inner,
-            static_cast<int>(cw), chunks);
-      else
-        strided_fwht_kernel<<<static_cast<unsigned>(blocks), 512,
-                              static_cast<size_t>(a * cw * 4), st>>>(
-            base + j * a * stride, so, static_cast<int>(a), stride, inner,
-            static_cast<int>(cw), chunks);
-      KQ_CHECK_LAUNCH();
-    }
-    // The next pass combines elements `a` positions apart; its independent
-    // vectors are (outer, position within this pass). They form one regular
-    // axis only when the outer axis tiles the current stride exactly.
-    if (A / a > 1) {
-      if (outer * so != stride) return KRONQ_ERR_UNSUPPORTED;
-      outer *= a;
-    }
-    stride *= a;
-    A /= a;
-  }
-  return KRONQ_OK;
+    const int64_t blocks = outer * n2 * chunks;
+    if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+    if (vec && cw % 4 == 0)
+      strided_fwht4_kernel<<<static_cast<unsigned>(blocks), 512,
+                             static_cast<size_t>(a * cw * 4), st>>>(
+          base, so, outer, so2, static_cast<int>(a), stride, inner,
+          static_cast<int>(cw), chunks);
+    else
+      strided_fwht_kernel<<<static_cast<unsigned>(blocks), 512,
+                            static_cast<size_t>(a * cw * 4), st>>>(
+          base, so, outer, so2, static_cast<int>(a), stride, inner,
+          static_cast<int>(cw), chunks);
+    KQ_CHECK_LAUNCH();
+    return KRONQ_OK;
+  };
+  if (A <= MAX_A) return pass(A, smid, 1, 0);
+  int64_t lo = 1;
+  while (lo * lo < A) lo *= 2;  // lo >= sqrt(A), both factors <= MAX_A
+  const int64_t hi = A / lo;
+  if (lo > MAX_A || hi > MAX_A) return KRONQ_ERR_UNSUPPORTED;
+  // low factor: elements smid apart; vectors (outer, high position)
+  KQ_TRY(pass(lo, smid, hi, lo * smid));
+  // high factor: elements lo*smid apart; vectors (outer, low position)
+  return pass(hi, lo * smid, lo, smid);
 }
 
 // out = P_r diag(cr) in diag(cc) P_cᵀ for an R x C row-major matrix.

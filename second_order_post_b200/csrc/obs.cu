@@ -25,8 +25,84 @@ constexpr int OROWS = (OTHREADS / 32) * RPW;
 constexpr int SUPER = 1024;    // super-block width
 constexpr int OSMEM = (OB * OB + OB) * 4;
 
-__device__ __forceinline__ float pick4(const float (&v)[4], int s) {
-  return s == 0 ? v[0] : s == 1 ? v[1] : s == 2 ? v[2] : v[3];
+// Columns [32*SLOT, 32*SLOT + 32) of the block for the warp's RPW rows. With
+// the register slot fixed at compile time, columns left of the chunk need no
+// update and columns right of it are updated without predicates.
+template <int SLOT>
+__device__ __forceinline__ void obs_chunk(float (&w)[RPW][4], float (&err)[RPW][4],
+                                          float (&scale)[RPW], float (&rscale)[RPW],
+                                          float (&zero)[RPW], const float *Us,
+                                          const float *inv, uint8_t (*qs)[OB],
+                                          int lane, int group, float maxq,
+                                          int64_t row0, int64_t d_out, int64_t j0,
+                                          float *scales, uint8_t *zeros,
+                                          int64_t ngroups) {
+  constexpr int jb = 32 * SLOT;
+  if (jb % group == 0) {
+    // group start: (scale, zero) from the rows' current weights of the group
+    float mn[RPW], mx[RPW];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      mn[r] = INFINITY;
+      mx[r] = -INFINITY;
+#pragma unroll
+      for (int s = SLOT; s < 4; ++s) {
+        if (32 * s < jb + group) {
+          mn[r] = fminf(mn[r], w[r][s]);
+          mx[r] = fmaxf(mx[r], w[r][s]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
+      }
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float xmin = fminf(mn[r], 0.f), xmax = fmaxf(mx[r], 0.f);
+      if (xmax == xmin) {
+        scale[r] = 1.f;
+        zero[r] = 0.f;
+      } else {
+        scale[r] = (xmax - xmin) / maxq;
+        zero[r] = rintf(-xmin / scale[r]);
+      }
+      rscale[r] = 1.f / scale[r];
+      if (lane == 0 && row0 + r < d_out) {
+        const int64_t gi = (j0 + jb) / group;
+        scales[(row0 + r) * ngroups + gi] = scale[r];
+        zeros[(row0 + r) * ngroups + gi] = static_cast<uint8_t>(zero[r]);
+      }
+    }
+  }
+  for (int jj = 0; jj < 32; ++jj) {
+    const int j = jb + jj;
+    const float *urow = Us + j * OB + lane;
+    float u[4];
+#pragma unroll
+    for (int s = SLOT; s < 4; ++s) u[s] = urow[32 * s];
+    const float iu = inv[j];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float wj = __shfl_sync(0xffffffffu, w[r][SLOT], jj);
+      // w/scale as a product with the group's reciprocal: it can differ from
+      // the quotient only within an ulp of a rounding tie
+      const float q = fminf(fmaxf(rintf(wj * rscale[r]) + zero[r], 0.f), maxq);
+      const float wh = scale[r] * (q - zero[r]);
+      const float e = (wj - wh) * iu;
+      if (lane > jj) w[r][SLOT] = fmaf(-e, u[SLOT], w[r][SLOT]);
+#pragma unroll
+      for (int s = SLOT + 1; s < 4; ++s) w[r][s] = fmaf(-e, u[s], w[r][s]);
+      if (lane == jj) {
+        w[r][SLOT] = wh;
+        err[r][SLOT] = e;
+        qs[r][j] = static_cast<uint8_t>(q);
+      }
+    }
+  }
 }
 
 // One 128-column block for OROWS rows per CTA. Each warp sweeps its 4 rows
@@ -63,71 +139,16 @@ __global__ void __launch_bounds__(OTHREADS)
       err[r][s] = 0.f;
     }
   }
-  float scale[RPW], zero[RPW];
-  for (int j = 0; j < OB; ++j) {
-    if (j % group == 0) {
-      float mn[RPW], mx[RPW];
-#pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        mn[r] = INFINITY;
-        mx[r] = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const int c = lane + 32 * s;
-          if (c >= j && c < j + group) {
-            mn[r] = fminf(mn[r], w[r][s]);
-            mx[r] = fmaxf(mx[r], w[r][s]);
-          }
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) {
-          mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
-          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
-        }
-#pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        const float xmin = fminf(mn[r], 0.f), xmax = fmaxf(mx[r], 0.f);
-        if (xmax == xmin) {
-          scale[r] = 1.f;
-          zero[r] = 0.f;
-        } else {
-          scale[r] = (xmax - xmin) / maxq;
-          zero[r] = rintf(-xmin / scale[r]);
-        }
-        if (lane == 0 && row0 + r < d_out) {
-          const int64_t gi = (j0 + j) / group;
-          scales[(row0 + r) * ngroups + gi] = scale[r];
-          zeros[(row0 + r) * ngroups + gi] = static_cast<uint8_t>(zero[r]);
-        }
-      }
-    }
-    const int slot = j >> 5, owner = j & 31;
-    const float *urow = Us + j * OB;
-    float u[4];
-#pragma unroll
-    for (int s = 0; s < 4; ++s) u[s] = urow[lane + 32 * s];
-    const float iu = inv[j];
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float wj = __shfl_sync(0xffffffffu, pick4(w[r], slot), owner);
-      const float q = fminf(fmaxf(rintf(wj / scale[r]) + zero[r], 0.f), maxq);
-      const float wh = scale[r] * (q - zero[r]);
-      const float e = (wj - wh) * iu;
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int c = lane + 32 * s;
-        if (c > j) w[r][s] = fmaf(-e, u[s], w[r][s]);
-        if (s == slot && lane == owner) {
-          w[r][s] = wh;
-          err[r][s] = e;
-        }
-      }
-      if (lane == owner) qsm[warp][r][j] = static_cast<uint8_t>(q);
-    }
-  }
+  float scale[RPW], rscale[RPW], zero[RPW];
+  uint8_t (*qs)[OB] = qsm[warp];
+  obs_chunk<0>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
+               d_out, j0, scales, zeros, ngroups);
+  obs_chunk<1>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
+               d_out, j0, scales, zeros, ngroups);
+  obs_chunk<2>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
+               d_out, j0, scales, zeros, ngroups);
+  obs_chunk<3>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
+               d_out, j0, scales, zeros, ngroups);
   __syncwarp();
   const int nwords = OB * bits / 32;
 #pragma unroll
