@@ -43,31 +43,48 @@ __global__ void damping_kernel(const float *H, int64_t d, float damp_rel,
   }
 }
 
-// Sweep-1 step for one row: row[k] -= colj[k*LP] * f for k = k0, k0+4, ... < j.
-// The row (A[i][k], k < j) and the pivot column (A[k][j]) never share an
-// element, so the loads can run ahead of the stores.
-__device__ __forceinline__ void ldl_row_step(float *__restrict__ row,
-                                             const float *__restrict__ colj,
-                                             int k0, int j, float f) {
-#pragma unroll 4
-  for (int k = k0; k < j; k += 4) row[k] = fmaf(-colj[k * LP], f, row[k]);
-}
-
 // One diagonal leaf at rows/cols [off, off+NB): reads the upper triangle of the
 // (already updated) block, adds λ, writes U (upper, zeros below).
-// Sweep 1, reverse LDLᵀ in shared memory: thread (row i, residue q) updates
-// A[i][k] for k ≡ q (mod 4); warps are numbered so that each scheduler holds
-// all four row blocks of one residue (balanced). One barrier per column.
-// Sweep 2, X = (unit upper)^-1 one column at a time from the bottom row up:
-// four lanes of a warp share a column and split the k-sum, no block barrier.
+//
+// Sweep 1, reverse LDLᵀ (H = Ŕ D Ŕᵀ, Ŕ unit upper), blocked by 32 columns from
+// the right; for each sub-block [c0, c0+32):
+//   (a) warp 0 factors the diagonal sub-block: lane l keeps row c0+l in
+//       registers, column entries of other rows arrive by shuffle;
+//   (b) one thread per row i < c0 applies the same 32 steps to its panel row;
+//   (c) all threads apply the rank-32 update of the leading block.
+// Sweep 2, X = Ŕ^-1: four warps invert the diagonal sub-blocks in parallel,
+// then the off-diagonal sub-blocks follow block diagonal by block diagonal
+// (X_IJ = -X_II Σ_K Ŕ_IK X_KJ) as small shared-memory products.
+constexpr int SB = 32;
+
+// C[32x32] = alpha * sum over terms of A_t[32x32] * B_t[32x32] for several
+// independent outputs at once (all operands in shared memory, pitch LP).
+struct BlkTerm {
+  const float *A, *B;
+};
+__device__ void small_products(int n_out, float **C, const BlkTerm (*terms)[3],
+                               const int *n_terms, float alpha) {
+  for (int e = threadIdx.x; e < n_out * SB * SB; e += blockDim.x) {
+    const int o = e / (SB * SB), r = (e / SB) % SB, c = e % SB;
+    float s = 0.f;
+    for (int t = 0; t < n_terms[o]; ++t) {
+      const float *a = terms[o][t].A + r * LP, *b = terms[o][t].B + c;
+#pragma unroll 8
+      for (int k = 0; k < SB; ++k) s = fmaf(a[k], b[k * LP], s);
+    }
+    C[o][r * LP + c] = alpha * s;
+  }
+}
+
 __global__ void __launch_bounds__(LTHREADS)
     chol_leaf_kernel(float *__restrict__ H, int64_t ld, int64_t off,
                      const float *__restrict__ lambda, int32_t *info) {
   extern __shared__ float sm[];
-  float *A = sm;                 // NB x LP
-  float *X = sm + NB * LP;       // NB x LP
-  float *piv = X + NB * LP;      // NB pivots
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  float *A = sm;                  // NB x LP: LDLᵀ, then the unit factor
+  float *X = A + NB * LP;         // NB x LP: inverse of the unit factor
+  float *T = X + NB * LP;         // 3 x SB x LP temporaries
+  float *piv = T + 3 * SB * LP;   // NB pivots
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const float lam = *lambda;
   for (int e = t; e < NB * NB; e += LTHREADS) {
     const int r = e / NB, c = e % NB;
@@ -78,54 +95,129 @@ __global__ void __launch_bounds__(LTHREADS)
     }
   }
   __syncthreads();
-  // ---- sweep 1
-  {
-    const int q = w & 3, i = 32 * (w >> 2) + lane;
-    const int k0 = i + ((q - i) & 3);  // first k >= i with k ≡ q (mod 4)
-    bool bad = false;
-    for (int j = NB - 1; j >= 0; --j) {
-      const float p = A[j * LP + j];
-      if (t == 0) {
-        piv[j] = p;
-        if (!(p > 0.f) || !isfinite(p)) {
-          if (!bad) report(info, KRONQ_ERR_NOT_PD | static_cast<int32_t>((off + j) << 8));
-          bad = true;
+  // ================= sweep 1
+  for (int J = NB / SB - 1; J >= 0; --J) {
+    const int c0 = SB * J;
+    if (warp == 0) {  // (a) diagonal sub-block, row c0+lane in registers
+      float r[SB];
+#pragma unroll
+      for (int k = 0; k < SB; ++k) r[k] = (k >= lane) ? A[(c0 + lane) * LP + c0 + k] : 0.f;
+      bool bad = false;
+#pragma unroll
+      for (int jj = SB - 1; jj >= 0; --jj) {
+        const float p = __shfl_sync(0xffffffffu, r[jj], jj);
+        if (lane == 0) {
+          piv[c0 + jj] = p;
+          if (!(p > 0.f) || !isfinite(p)) {
+            if (!bad) report(info, KRONQ_ERR_NOT_PD | static_cast<int32_t>((off + c0 + jj) << 8));
+            bad = true;
+          }
+        }
+        const float f = r[jj] / p;
+#pragma unroll
+        for (int k = 0; k < jj; ++k) {
+          const float ck = __shfl_sync(0xffffffffu, r[jj], k);  // A[c0+k][c0+jj]
+          if (lane <= k && lane < jj) r[k] = fmaf(-ck, f, r[k]);
         }
       }
-      if (i < j) ldl_row_step(A + i * LP, A + j, k0, j, A[i * LP + j] / p);
-      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < SB; ++k)
+        if (k >= lane) A[(c0 + lane) * LP + c0 + k] = r[k];
     }
+    __syncthreads();
+    if (c0 == 0) break;
+    if (t < c0) {  // (b) panel row t: A[t][c0 .. c0+31]
+      float q[SB];
+      float *row = A + t * LP + c0;
+#pragma unroll
+      for (int k = 0; k < SB; ++k) q[k] = row[k];
+#pragma unroll
+      for (int jj = SB - 1; jj >= 0; --jj) {
+        const float f = q[jj] / piv[c0 + jj];
+#pragma unroll
+        for (int k = 0; k < jj; ++k) q[k] = fmaf(-A[(c0 + k) * LP + c0 + jj], f, q[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < SB; ++k) row[k] = q[k];
+    }
+    __syncthreads();
+    {  // (c) A[i][k] -= sum_jj A[i][c0+jj] A[k][c0+jj] / piv[c0+jj], i <= k < c0
+      const int k = t % NB, r0 = t / NB;
+      if (k < c0) {
+        float g[SB];
+#pragma unroll
+        for (int jj = 0; jj < SB; ++jj) g[jj] = A[k * LP + c0 + jj] / piv[c0 + jj];
+        for (int i = r0; i <= k; i += LTHREADS / NB) {
+          const float *ri = A + i * LP + c0;
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < SB; jj += 2) {
+            s0 = fmaf(ri[jj], g[jj], s0);
+            s1 = fmaf(ri[jj + 1], g[jj + 1], s1);
+          }
+          A[i * LP + k] -= s0 + s1;
+        }
+      }
+    }
+    __syncthreads();
   }
-  // unit upper factor in place: A[i][k] / piv[k], i < k
+  // unit factor Ŕ[i][k] = A[i][k] / piv[k] (i < k); X = 0
   for (int e = t; e < NB * NB; e += LTHREADS) {
     const int r = e / NB, c = e % NB;
     if (c > r) A[r * LP + c] /= piv[c];
+    X[r * LP + c] = 0.f;
   }
   __syncthreads();
-  // ---- sweep 2: column c of X, lanes 4g..4g+3 of a warp share c
-  {
-    const int part = lane & 3;
-    const int c = 8 * w + (lane >> 2);
-    X[c * LP + c] = 1.f;  // X stored transposed: X[c][i] holds X(i, c)
-    __syncwarp();
-    float *xc = X + c * LP;
-    for (int i = NB - 2; i >= 0; --i) {
+  // ================= sweep 2
+  if (warp < NB / SB) {  // diagonal inverses, lane = column c0+lane
+    const int c0 = SB * warp;
+    float x[SB];
+#pragma unroll
+    for (int i = 0; i < SB; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = SB - 2; i >= 0; --i) {
       float s = 0.f;
-      if (i < c) {
-        const float *ri = A + i * LP;
-        for (int k = i + 1 + part; k <= c; k += 4) s = fmaf(ri[k], xc[k], s);
-      }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (part == 0 && i < c) xc[i] = -s;
-      __syncwarp();
+#pragma unroll
+      for (int k = i + 1; k < SB; ++k)
+        if (k <= lane) s = fmaf(A[(c0 + i) * LP + c0 + k], x[k], s);
+      if (i < lane) x[i] = -s;
     }
+#pragma unroll
+    for (int i = 0; i < SB; ++i)
+      if (i <= lane) X[(c0 + i) * LP + c0 + lane] = x[i];
   }
   __syncthreads();
+  for (int dist = 1; dist < NB / SB; ++dist) {
+    const int n = NB / SB - dist;  // blocks (I, I+dist), I < n
+    float *Cs[3];
+    BlkTerm terms[3][3];
+    int nt[3];
+    // T_I = sum_{K=I+1..J} Ŕ_IK X_KJ
+    for (int I = 0; I < n; ++I) {
+      const int J = I + dist;
+      Cs[I] = T + I * SB * LP;
+      nt[I] = dist;
+      for (int m = 0; m < dist; ++m) {
+        const int K = I + 1 + m;
+        terms[I][m] = {A + (SB * I) * LP + SB * K, X + (SB * K) * LP + SB * J};
+      }
+    }
+    small_products(n, Cs, terms, nt, 1.f);
+    __syncthreads();
+    // X_IJ = -X_II T_I
+    for (int I = 0; I < n; ++I) {
+      const int J = I + dist;
+      Cs[I] = X + (SB * I) * LP + SB * J;
+      nt[I] = 1;
+      terms[I][0] = {X + (SB * I) * LP + SB * I, T + I * SB * LP};
+    }
+    small_products(n, Cs, terms, nt, -1.f);
+    __syncthreads();
+  }
   // U(i, c) = X(i, c) / sqrt(piv[i]) for i <= c, zeros below the diagonal
   for (int e = t; e < NB * NB; e += LTHREADS) {
     const int i = e / NB, c = e % NB;
-    H[(off + i) * ld + off + c] = (i <= c) ? X[c * LP + i] / sqrtf(piv[i]) : 0.f;
+    H[(off + i) * ld + off + c] = (i <= c) ? X[i * LP + c] / sqrtf(piv[i]) : 0.f;
   }
 }
 
@@ -150,7 +242,7 @@ struct Ctx {
 inline int64_t first_half(int64_t n) { return (n / NB / 2) * NB; }
 
 kronq_status leaf(const Ctx &c, int64_t off) {
-  const int smem = (2 * NB * LP + NB) * sizeof(float);
+  const int smem = (2 * NB * LP + 3 * SB * LP + NB) * sizeof(float);
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(chol_leaf_kernel,
