@@ -12,17 +12,17 @@
 //     U12 = -U11 (V U22)
 // All off-diagonal work runs as fp32-accurate 3xTF32 tcgen05 GEMMs that skip
 // the zero blocks of the triangular operands; 128x128 diagonal leaves are
-// factored in shared memory by one CTA. λ = damp_rel * mean(diag H) is added
+// factored and inverted in registers by one CTA. λ = damp_rel * mean(diag H) is added
 // by each leaf to its own diagonal (the updates never touch λ, so this equals
 // damping H up front).
+#include <mutex>
+
 #include "kernels.cuh"
 
 namespace kronq {
 namespace {
 
 constexpr int NB = 128;
-constexpr int LP = NB + 1;  // padded pitch of the leaf tiles
-constexpr int LTHREADS = 512;
 
 __global__ void damping_kernel(const float *H, int64_t d, float damp_rel,
                                float *lambda, int32_t *info) {
@@ -46,178 +46,182 @@ __global__ void damping_kernel(const float *H, int64_t d, float damp_rel,
 // One diagonal leaf at rows/cols [off, off+NB): reads the upper triangle of the
 // (already updated) block, adds λ, writes U (upper, zeros below).
 //
-// Sweep 1, reverse LDLᵀ (H = Ŕ D Ŕᵀ, Ŕ unit upper), blocked by 32 columns from
-// the right; for each sub-block [c0, c0+32):
-//   (a) warp 0 factors the diagonal sub-block: lane l keeps row c0+l in
-//       registers, column entries of other rows arrive by shuffle;
-//   (b) one thread per row i < c0 applies the same 32 steps to its panel row;
-//   (c) all threads apply the rank-32 update of the leading block.
-// Sweep 2, X = Ŕ^-1: four warps invert the diagonal sub-blocks in parallel,
-// then the off-diagonal sub-blocks follow block diagonal by block diagonal
-// (X_IJ = -X_II Σ_K Ŕ_IK X_KJ) as small shared-memory products.
-constexpr int SB = 32;
-
-// C[32x32] = alpha * sum over terms of A_t[32x32] * B_t[32x32] for several
-// independent outputs at once (all operands in shared memory, pitch LP).
-struct BlkTerm {
-  const float *A, *B;
-};
-__device__ void small_products(int n_out, float **C, const BlkTerm (*terms)[3],
-                               const int *n_terms, float alpha) {
-  for (int e = threadIdx.x; e < n_out * SB * SB; e += blockDim.x) {
-    const int o = e / (SB * SB), r = (e / SB) % SB, c = e % SB;
-    float s = 0.f;
-    for (int t = 0; t < n_terms[o]; ++t) {
-      const float *a = terms[o][t].A + r * LP, *b = terms[o][t].B + c;
-#pragma unroll 8
-      for (int k = 0; k < SB; ++k) s = fmaf(a[k], b[k * LP], s);
-    }
-    C[o][r * LP + c] = alpha * s;
-  }
-}
+// Factor and inverse come out of one sweep over the pivots jj = NB-1 .. 0.
+// With H = Ŕ D Ŕᵀ (Ŕ unit upper, columns l_j above the diagonal),
+// Ŕ = (I + l_{NB-1} e_{NB-1}ᵀ) ... (I + l_0 e_0ᵀ), so X = Ŕ^-1 is the product of
+// (I - l_j e_jᵀ) taken from j = 0 on the left to j = NB-1 on the right; pivot jj
+// contributes the left factor X <- (I - l_jj e_jjᵀ) X, a rank-1 update of the
+// rows above jj, and row jj of X is final when pivot jj is taken. One array M
+// holds the Schur complement left of the current column and X from it on, and
+// pivot jj applies to every row i < jj and column k >= i
+//     M[i][k] -= l[i] * b[k],  l[i] = M[i][jj] / p,
+//     b[k] = M[k][jj] (k < jj),  p + 1 (k = jj),  M[jj][k] (k > jj),
+// which is the Schur update left of jj, turns column jj into -l, and applies
+// the left factor right of it. U = D^-1/2 X.
+//
+// Each thread keeps one 4x4 tile of the upper triangle in registers. Pivots
+// are taken four at a time (the pivot block J = [j0, j0+4) is one tile): the
+// owners of tile column J publish their tiles (M[i][J], i < j0+4, the pivot
+// block included) and the owners of tile row J theirs (M[J][k], k >= j0+4),
+// and after one barrier every thread replays the four pivots on its own tile.
+// Within the block, pivot jj changes the published values that later pivots
+// of the block read; each thread carries those along itself:
+//     M[i][j'] -= (M[i][jj] / p) M[j'][jj]      (its rows, j' < jj in J)
+//     b_j'[k]  -= (M[j'][jj] / p) b_jj[k]        (its columns outside J)
+// and factors the 4x4 pivot block redundantly, so a block costs one barrier.
+constexpr int TT = 4;                          // tile edge owned by a thread
+constexpr int NT = NB / TT;                    // tile rows and columns
+constexpr int NTILES = NT * (NT + 1) / 2;      // upper tiles (I <= K)
+constexpr int LTHREADS = (NTILES + 31) / 32 * 32;
 
 __global__ void __launch_bounds__(LTHREADS)
     chol_leaf_kernel(float *__restrict__ H, int64_t ld, int64_t off,
                      const float *__restrict__ lambda, int32_t *info) {
-  extern __shared__ float sm[];
-  float *A = sm;                  // NB x LP: LDLᵀ, then the unit factor
-  float *X = A + NB * LP;         // NB x LP: inverse of the unit factor
-  float *T = X + NB * LP;         // 3 x SB x LP temporaries
-  float *piv = T + 3 * SB * LP;   // NB pivots
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const float lam = *lambda;
-  for (int e = t; e < NB * NB; e += LTHREADS) {
-    const int r = e / NB, c = e % NB;
-    if (c >= r) {
-      float v = H[(off + r) * ld + off + c];
-      if (c == r) v += lam;
-      A[r * LP + c] = v;
+  __shared__ __align__(16) float colbuf[2][NB][TT];  // M[i][J], row i
+  __shared__ __align__(16) float rowbuf[2][TT][NB];  // M[J][k]
+  __shared__ float piv[NB];
+  const int t = threadIdx.x;
+  const bool own = t < NTILES;
+  int I = NT, K = NT;  // tile of this thread, row-major over the upper tiles
+  if (own) {
+    int r = t;
+    I = 0;
+    while (r >= NT - I) {
+      r -= NT - I;
+      ++I;
+    }
+    K = I + r;
+  }
+  const int r0 = TT * I, c0 = TT * K;
+  float m[TT][TT];
+  if (own) {
+    const float lam = *lambda;
+#pragma unroll
+    for (int ii = 0; ii < TT; ++ii) {
+      const float4 v =
+          *reinterpret_cast<const float4 *>(H + (off + r0 + ii) * ld + off + c0);
+      m[ii][0] = v.x; m[ii][1] = v.y; m[ii][2] = v.z; m[ii][3] = v.w;
+      if (I == K) {
+#pragma unroll
+        for (int kk = 0; kk < TT; ++kk) {
+          if (kk < ii) m[ii][kk] = 0.f;
+          if (kk == ii) m[ii][kk] += lam;
+        }
+      }
     }
   }
+  auto publish = [&](int Tj) {
+    if (K == Tj) {
+#pragma unroll
+      for (int ii = 0; ii < TT; ++ii)
+        *reinterpret_cast<float4 *>(&colbuf[Tj & 1][r0 + ii][0]) =
+            make_float4(m[ii][0], m[ii][1], m[ii][2], m[ii][3]);
+    } else if (I == Tj) {
+#pragma unroll
+      for (int ii = 0; ii < TT; ++ii)
+        *reinterpret_cast<float4 *>(&rowbuf[Tj & 1][ii][c0]) =
+            make_float4(m[ii][0], m[ii][1], m[ii][2], m[ii][3]);
+    }
+  };
+  if (own) publish(NT - 1);
   __syncthreads();
-  // ================= sweep 1
-  for (int J = NB / SB - 1; J >= 0; --J) {
-    const int c0 = SB * J;
-    if (warp == 0) {  // (a) diagonal sub-block, row c0+lane in registers
-      float r[SB];
+  bool bad = false;
+  for (int Tj = NT - 1; Tj >= 0; --Tj) {
+    const int j0 = TT * Tj, bs_ = Tj & 1;
+    if (own && I <= Tj) {
+      float blk[TT][TT], ar[TT][TT], bsrc[TT][TT];
 #pragma unroll
-      for (int k = 0; k < SB; ++k) r[k] = (k >= lane) ? A[(c0 + lane) * LP + c0 + k] : 0.f;
-      bool bad = false;
+      for (int a = 0; a < TT; ++a) {
+        const float4 v = *reinterpret_cast<const float4 *>(&colbuf[bs_][j0 + a][0]);
+        blk[a][0] = v.x; blk[a][1] = v.y; blk[a][2] = v.z; blk[a][3] = v.w;
+        const float4 w = *reinterpret_cast<const float4 *>(&colbuf[bs_][r0 + a][0]);
+        ar[a][0] = w.x; ar[a][1] = w.y; ar[a][2] = w.z; ar[a][3] = w.w;
+      }
+      const bool in_blk = K == Tj;
+      if (K < Tj) {  // columns left of J: b_jj[k] = M[k][jj]
 #pragma unroll
-      for (int jj = SB - 1; jj >= 0; --jj) {
-        const float p = __shfl_sync(0xffffffffu, r[jj], jj);
-        if (lane == 0) {
-          piv[c0 + jj] = p;
+        for (int kk = 0; kk < TT; ++kk) {
+          const float4 v = *reinterpret_cast<const float4 *>(&colbuf[bs_][c0 + kk][0]);
+          bsrc[0][kk] = v.x; bsrc[1][kk] = v.y; bsrc[2][kk] = v.z; bsrc[3][kk] = v.w;
+        }
+      } else if (K > Tj) {  // columns right of J: b_jj[k] = M[jj][k]
+#pragma unroll
+        for (int q = 0; q < TT; ++q) {
+          const float4 v = *reinterpret_cast<const float4 *>(&rowbuf[bs_][q][c0]);
+          bsrc[q][0] = v.x; bsrc[q][1] = v.y; bsrc[q][2] = v.z; bsrc[q][3] = v.w;
+        }
+      }
+#pragma unroll
+      for (int q = TT - 1; q >= 0; --q) {
+        const float p = blk[q][q];
+        const float rp = __frcp_rn(p);
+        if (t == 0) {
+          piv[j0 + q] = p;
           if (!(p > 0.f) || !isfinite(p)) {
-            if (!bad) report(info, KRONQ_ERR_NOT_PD | static_cast<int32_t>((off + c0 + jj) << 8));
+            if (!bad)
+              report(info, KRONQ_ERR_NOT_PD | static_cast<int32_t>((off + j0 + q) << 8));
             bad = true;
           }
         }
-        const float f = r[jj] / p;
+        float l[TT], b[TT];
 #pragma unroll
-        for (int k = 0; k < jj; ++k) {
-          const float ck = __shfl_sync(0xffffffffu, r[jj], k);  // A[c0+k][c0+jj]
-          if (lane <= k && lane < jj) r[k] = fmaf(-ck, f, r[k]);
-        }
-      }
+        for (int ii = 0; ii < TT; ++ii) l[ii] = r0 + ii < j0 + q ? ar[ii][q] * rp : 0.f;
 #pragma unroll
-      for (int k = 0; k < SB; ++k)
-        if (k >= lane) A[(c0 + lane) * LP + c0 + k] = r[k];
-    }
-    __syncthreads();
-    if (c0 == 0) break;
-    if (t < c0) {  // (b) panel row t: A[t][c0 .. c0+31]
-      float q[SB];
-      float *row = A + t * LP + c0;
+        for (int kk = 0; kk < TT; ++kk)
+          b[kk] = in_blk ? (kk < q ? blk[kk][q] : kk == q ? p + 1.f : blk[q][kk])
+                         : bsrc[q][kk];
 #pragma unroll
-      for (int k = 0; k < SB; ++k) q[k] = row[k];
+        for (int ii = 0; ii < TT; ++ii)
 #pragma unroll
-      for (int jj = SB - 1; jj >= 0; --jj) {
-        const float f = q[jj] / piv[c0 + jj];
+          for (int kk = 0; kk < TT; ++kk) m[ii][kk] = fmaf(-l[ii], b[kk], m[ii][kk]);
+        // carry the pivot into the values that the later pivots q' < q read
 #pragma unroll
-        for (int k = 0; k < jj; ++k) q[k] = fmaf(-A[(c0 + k) * LP + c0 + jj], f, q[k]);
-      }
+        for (int qq = 0; qq < q; ++qq) {
+          const float c = blk[qq][q] * rp;
 #pragma unroll
-      for (int k = 0; k < SB; ++k) row[k] = q[k];
-    }
-    __syncthreads();
-    {  // (c) A[i][k] -= sum_jj A[i][c0+jj] A[k][c0+jj] / piv[c0+jj], i <= k < c0
-      const int k = t % NB, r0 = t / NB;
-      if (k < c0) {
-        float g[SB];
+          for (int ii = 0; ii < TT; ++ii) ar[ii][qq] = fmaf(-ar[ii][q] * rp, blk[qq][q], ar[ii][qq]);
+          if (!in_blk) {
 #pragma unroll
-        for (int jj = 0; jj < SB; ++jj) g[jj] = A[k * LP + c0 + jj] / piv[c0 + jj];
-        for (int i = r0; i <= k; i += LTHREADS / NB) {
-          const float *ri = A + i * LP + c0;
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < SB; jj += 2) {
-            s0 = fmaf(ri[jj], g[jj], s0);
-            s1 = fmaf(ri[jj + 1], g[jj + 1], s1);
+            for (int kk = 0; kk < TT; ++kk) bsrc[qq][kk] = fmaf(-c, bsrc[q][kk], bsrc[qq][kk]);
           }
-          A[i * LP + k] -= s0 + s1;
+        }
+        float colq[TT], rowq[TT];
+#pragma unroll
+        for (int a = 0; a < TT; ++a) {
+          colq[a] = blk[a][q];
+          rowq[a] = blk[q][a];
+        }
+#pragma unroll
+        for (int a = 0; a < q; ++a) {
+          const float la = colq[a] * rp;
+#pragma unroll
+          for (int bb = a; bb < TT; ++bb) {
+            const float v = bb < q ? colq[bb] : bb == q ? p + 1.f : rowq[bb];
+            blk[a][bb] = fmaf(-la, v, blk[a][bb]);
+          }
         }
       }
     }
+    if (own && Tj > 0) publish(Tj - 1);
     __syncthreads();
   }
-  // unit factor Ŕ[i][k] = A[i][k] / piv[k] (i < k); X = 0
-  for (int e = t; e < NB * NB; e += LTHREADS) {
-    const int r = e / NB, c = e % NB;
-    if (c > r) A[r * LP + c] /= piv[c];
-    X[r * LP + c] = 0.f;
-  }
-  __syncthreads();
-  // ================= sweep 2
-  if (warp < NB / SB) {  // diagonal inverses, lane = column c0+lane
-    const int c0 = SB * warp;
-    float x[SB];
+  if (own) {
 #pragma unroll
-    for (int i = 0; i < SB; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+    for (int ii = 0; ii < TT; ++ii) {
+      const int i = r0 + ii;
+      const float s = 1.f / sqrtf(piv[i]);
+      float o[TT];
 #pragma unroll
-    for (int i = SB - 2; i >= 0; --i) {
-      float s = 0.f;
-#pragma unroll
-      for (int k = i + 1; k < SB; ++k)
-        if (k <= lane) s = fmaf(A[(c0 + i) * LP + c0 + k], x[k], s);
-      if (i < lane) x[i] = -s;
-    }
-#pragma unroll
-    for (int i = 0; i < SB; ++i)
-      if (i <= lane) X[(c0 + i) * LP + c0 + lane] = x[i];
-  }
-  __syncthreads();
-  for (int dist = 1; dist < NB / SB; ++dist) {
-    const int n = NB / SB - dist;  // blocks (I, I+dist), I < n
-    float *Cs[3];
-    BlkTerm terms[3][3];
-    int nt[3];
-    // T_I = sum_{K=I+1..J} Ŕ_IK X_KJ
-    for (int I = 0; I < n; ++I) {
-      const int J = I + dist;
-      Cs[I] = T + I * SB * LP;
-      nt[I] = dist;
-      for (int m = 0; m < dist; ++m) {
-        const int K = I + 1 + m;
-        terms[I][m] = {A + (SB * I) * LP + SB * K, X + (SB * K) * LP + SB * J};
+      for (int kk = 0; kk < TT; ++kk) {
+        const int k = c0 + kk;
+        o[kk] = k > i ? m[ii][kk] * s : (k == i ? s : 0.f);
       }
+      *reinterpret_cast<float4 *>(H + (off + i) * ld + off + c0) =
+          make_float4(o[0], o[1], o[2], o[3]);
+      if (I != K)  // mirrored tile below the diagonal
+        *reinterpret_cast<float4 *>(H + (off + c0 + ii) * ld + off + r0) =
+            make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    small_products(n, Cs, terms, nt, 1.f);
-    __syncthreads();
-    // X_IJ = -X_II T_I
-    for (int I = 0; I < n; ++I) {
-      const int J = I + dist;
-      Cs[I] = X + (SB * I) * LP + SB * J;
-      nt[I] = 1;
-      terms[I][0] = {X + (SB * I) * LP + SB * I, T + I * SB * LP};
-    }
-    small_products(n, Cs, terms, nt, -1.f);
-    __syncthreads();
-  }
-  // U(i, c) = X(i, c) / sqrt(piv[i]) for i <= c, zeros below the diagonal
-  for (int e = t; e < NB * NB; e += LTHREADS) {
-    const int i = e / NB, c = e % NB;
-    H[(off + i) * ld + off + c] = (i <= c) ? X[i * LP + c] / sqrtf(piv[i]) : 0.f;
   }
 }
 
@@ -228,30 +232,62 @@ __global__ void zero_lower_kernel(float *H, int64_t d) {
     H[r * d + c] = 0.f;
 }
 
+constexpr int MAXD = 40;  // recursion depth bound (d <= 65536 gives <= 10)
+
 struct Ctx {
-  cudaStream_t st;
+  cudaStream_t st;           // critical path (leaves, V, SYRK, U12)
+  cudaStream_t side[MAXD];   // T = V U22 of the node at each depth
+  cudaEvent_t ev_v[MAXD], ev_t[MAXD];
   float *H;
   int64_t d;
-  float *V;              // B U22ᵀ of the current node (dead before recursing)
-  float *T[40];          // V U22 of the node at each depth (kept across the
-                         // recursion into A11)
+  float *V[MAXD];            // B U22ᵀ of the node at each depth
+  float *T[MAXD];            // V U22 of the node at each depth
   const float *lambda;
   int32_t *info;
 };
 
+// Streams and events of the recursion, created once per device: the critical
+// path runs on a highest-priority stream so that its single-CTA leaves take
+// the next free SM ahead of the concurrent T products.
+struct CholStreams {
+  bool ready = false;
+  cudaStream_t main;
+  cudaStream_t side[MAXD];
+  cudaEvent_t ev_v[MAXD], ev_t[MAXD], fork, join_main, join_side[MAXD];
+};
+
+kronq_status chol_streams(CholStreams **out) {
+  static CholStreams per_dev[64];
+  static std::mutex mu;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KRONQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  CholStreams &cs = per_dev[dev];
+  if (!cs.ready) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return KRONQ_ERR_CUDA;
+    if (cudaStreamCreateWithPriority(&cs.main, cudaStreamNonBlocking, hi) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&cs.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&cs.join_main, cudaEventDisableTiming) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    for (int k = 0; k < MAXD; ++k) {
+      if (cudaStreamCreateWithPriority(&cs.side[k], cudaStreamNonBlocking, lo) != cudaSuccess ||
+          cudaEventCreateWithFlags(&cs.ev_v[k], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&cs.ev_t[k], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&cs.join_side[k], cudaEventDisableTiming) != cudaSuccess)
+        return KRONQ_ERR_CUDA;
+    }
+    cs.ready = true;
+  }
+  *out = &cs;
+  return KRONQ_OK;
+}
+
 inline int64_t first_half(int64_t n) { return (n / NB / 2) * NB; }
 
 kronq_status leaf(const Ctx &c, int64_t off) {
-  const int smem = (2 * NB * LP + 3 * SB * LP + NB) * sizeof(float);
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(chol_leaf_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr_done = true;
-  }
-  chol_leaf_kernel<<<1, LTHREADS, smem, c.st>>>(c.H, c.d, off, c.lambda, c.info);
+  chol_leaf_kernel<<<1, LTHREADS, 0, c.st>>>(c.H, c.d, off, c.lambda, c.info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
@@ -264,37 +300,45 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
   float *A11 = c.H + off * d + off;
   float *B12 = c.H + off * d + off + h;
   float *C22 = c.H + (off + h) * d + off + h;
-  float *T = c.T[depth];
+  if (depth >= MAXD - 1) return KRONQ_ERR_UNSUPPORTED;
+  float *V = c.V[depth], *T = c.T[depth];
   KQ_TRY(rinv(c, off + h, m, depth + 1));  // C22 -> U22
   {
     GemmArgs g;  // V = B U22ᵀ : V[i][j] = sum_k B[i][k] U22[j][k], k >= j
     g.M = h; g.N = m; g.K = m;
     g.A = B12; g.lda = d;
     g.B = C22; g.ldb = d;
-    g.C = c.V; g.ldc = m;
+    g.C = V; g.ldc = m;
     g.kflags = KR_B_UPPER;
     KQ_TRY(gemm_tf32x3(c.st, g, c.info));
   }
+  // T = V U22 does not feed the recursion into A11: run it beside it
+  if (cudaEventRecord(c.ev_v[depth], c.st) != cudaSuccess ||
+      cudaStreamWaitEvent(c.side[depth], c.ev_v[depth], 0) != cudaSuccess)
+    return KRONQ_ERR_CUDA;
+  {
+    GemmArgs g;  // T = V U22 : T[i][j] = sum_k V[i][k] U22[k][j], k <= j
+    g.M = h; g.N = m; g.K = m;
+    g.A = V; g.lda = m;
+    g.B = C22; g.ldb = d; g.b_mn = true;
+    g.C = T; g.ldc = m;
+    g.kflags = KR_B_LOWER;
+    KQ_TRY(gemm_tf32x3(c.side[depth], g, c.info));
+  }
+  if (cudaEventRecord(c.ev_t[depth], c.side[depth]) != cudaSuccess)
+    return KRONQ_ERR_CUDA;
   {
     GemmArgs g;  // A11 -= V Vᵀ (tiles on or above the diagonal)
     g.M = h; g.N = h; g.K = m;
-    g.A = c.V; g.lda = m;
-    g.B = c.V; g.ldb = m;
+    g.A = V; g.lda = m;
+    g.B = V; g.ldb = m;
     g.C = A11; g.ldc = d;
     g.alpha = -1.f; g.beta = 1.f;
     g.upper_tiles_only = true;
     KQ_TRY(gemm_tf32x3(c.st, g, c.info));
   }
-  {
-    GemmArgs g;  // T = V U22 : T[i][j] = sum_k V[i][k] U22[k][j], k <= j
-    g.M = h; g.N = m; g.K = m;
-    g.A = c.V; g.lda = m;
-    g.B = C22; g.ldb = d; g.b_mn = true;
-    g.C = T; g.ldc = m;
-    g.kflags = KR_B_LOWER;
-    KQ_TRY(gemm_tf32x3(c.st, g, c.info));
-  }
   KQ_TRY(rinv(c, off, h, depth + 1));  // A11 -> U11
+  if (cudaStreamWaitEvent(c.st, c.ev_t[depth], 0) != cudaSuccess) return KRONQ_ERR_CUDA;
   {
     GemmArgs g;  // U12 = -U11 T : U11[i][k] == 0 for k < i
     g.M = h; g.N = m; g.K = h;
@@ -308,17 +352,18 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
   return KRONQ_OK;
 }
 
-// Workspace layout: [V: h0*m0][T slot per depth][lambda]. The largest node at
-// depth i+1 is the larger child m_i of the largest node at depth i.
-size_t chol_layout(int64_t d, size_t *t_off, int *depths) {
+// Workspace layout: [V slot, T slot] per recursion depth, then lambda. The
+// largest node at depth i+1 is the larger child m_i of the largest node at i.
+size_t chol_layout(int64_t d, size_t *v_off, size_t *t_off, int *depths) {
   auto al = [](size_t b) { return (b + 255) / 256 * 256; };
-  const int64_t h0 = first_half(d);
-  size_t off = al(static_cast<size_t>(h0) * (d - h0) * 4);
+  size_t off = 0;
   int k = 0;
-  for (int64_t n = d; n > NB && k < 40; ++k) {
+  for (int64_t n = d; n > NB && k < MAXD; ++k) {
     const int64_t h = first_half(n);
-    if (t_off) t_off[k] = off;
-    off += al(static_cast<size_t>(h) * (n - h) * 4);
+    const size_t slot = al(static_cast<size_t>(h) * (n - h) * 4);
+    if (v_off) v_off[k] = off;
+    if (t_off) t_off[k] = off + slot;
+    off += 2 * slot;
     n = n - h;
   }
   if (depths) *depths = k;
@@ -327,32 +372,53 @@ size_t chol_layout(int64_t d, size_t *t_off, int *depths) {
 
 }  // namespace
 
-size_t chol_ws_bytes(int64_t d) { return chol_layout(d, nullptr, nullptr); }
+size_t chol_ws_bytes(int64_t d) { return chol_layout(d, nullptr, nullptr, nullptr); }
 
 kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
                       void *ws, size_t ws_bytes, int32_t *info) {
-  size_t t_off[40];
+  size_t v_off[MAXD], t_off[MAXD];
   int depths = 0;
-  const size_t need = chol_layout(d, t_off, &depths);
+  const size_t need = chol_layout(d, v_off, t_off, &depths);
   if (ws_bytes < need) return KRONQ_ERR_INVALID_ARG;
+  CholStreams *cs = nullptr;
+  KQ_TRY(chol_streams(&cs));
   uint8_t *w = static_cast<uint8_t *>(ws);
   Ctx c;
-  c.st = st;
+  c.st = cs->main;
   c.H = H;
   c.d = d;
-  c.V = reinterpret_cast<float *>(w);
-  for (int k = 0; k < 40; ++k)
+  for (int k = 0; k < MAXD; ++k) {
+    c.side[k] = cs->side[k];
+    c.ev_v[k] = cs->ev_v[k];
+    c.ev_t[k] = cs->ev_t[k];
+    c.V[k] = k < depths ? reinterpret_cast<float *>(w + v_off[k]) : nullptr;
     c.T[k] = k < depths ? reinterpret_cast<float *>(w + t_off[k]) : nullptr;
+  }
   float *lambda = reinterpret_cast<float *>(w + need - 256);
   c.lambda = lambda;
   c.info = info;
-  damping_kernel<<<1, 1024, 0, st>>>(H, d, damp_rel, lambda, info);
+  // fork from the caller's stream
+  if (cudaEventRecord(cs->fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(cs->main, cs->fork, 0) != cudaSuccess)
+    return KRONQ_ERR_CUDA;
+  for (int k = 0; k < depths; ++k)
+    if (cudaStreamWaitEvent(cs->side[k], cs->fork, 0) != cudaSuccess) return KRONQ_ERR_CUDA;
+  damping_kernel<<<1, 1024, 0, c.st>>>(H, d, damp_rel, lambda, info);
   KQ_CHECK_LAUNCH();
   KQ_TRY(rinv(c, 0, d, 0));
   dim3 grid(static_cast<unsigned>(kq_min<int64_t>(ceil_div(d, 256), 64)),
             static_cast<unsigned>(d));
-  zero_lower_kernel<<<grid, 256, 0, st>>>(H, d);
+  zero_lower_kernel<<<grid, 256, 0, c.st>>>(H, d);
   KQ_CHECK_LAUNCH();
+  // join back into the caller's stream (every side stream is idle by now
+  // from the main stream's point of view; joining them keeps ws reuse safe)
+  if (cudaEventRecord(cs->join_main, cs->main) != cudaSuccess ||
+      cudaStreamWaitEvent(st, cs->join_main, 0) != cudaSuccess)
+    return KRONQ_ERR_CUDA;
+  for (int k = 0; k < depths; ++k)
+    if (cudaEventRecord(cs->join_side[k], cs->side[k]) != cudaSuccess ||
+        cudaStreamWaitEvent(st, cs->join_side[k], 0) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
   return KRONQ_OK;
 }
 
