@@ -267,6 +267,26 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
                               const float *H_G, int64_t d_out, int64_t d_in,
                               double *loss_dev, void *ws, size_t ws_bytes);
 
+/*
+ * fp32-accurate dense product on the tensor cores (the contraction behind the
+ * Cholesky recursion, the OBS trailing updates and the layer loss; the pages
+ * name no such routine): C = alpha * A * B^T + beta * C with row-major
+ * operands on the device,
+ *   A: M x K (a_mn = 0, pitch lda) or its transpose stored K x M (a_mn = 1),
+ *   B: N x K (b_mn = 0, pitch ldb) or its transpose stored K x N (b_mn = 1),
+ *   C: M x N, pitch ldc; beta = 0 ignores the old C.
+ * Each fp32 operand is split into TF32 high and low parts and three MMAs
+ * (hi*hi, hi*lo, lo*hi) accumulate in fp32. Pointers 16-byte aligned,
+ * pitches multiples of 4 elements; M, N, K >= 0. C must not overlap A or B.
+ * INVALID_ARG for negative sizes or null pointers, UNSUPPORTED for
+ * misaligned operands, TIMEOUT in *info_dev (nonzero) if a pipeline wait
+ * ran out.
+ */
+kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,
+                            int64_t K, float alpha, const float *A, int64_t lda,
+                            int a_mn, const float *B, int64_t ldb, int b_mn,
+                            float beta, float *C, int64_t ldc, int32_t *info_dev);
+
 /* Workspace bytes needed by one call (opts may be NULL except for BIIP and
  * QUANT). Returns 0 for unsupported arguments. */
 size_t kronq_workspace_bytes(kronq_ws_kind which, int64_t d_out, int64_t d_in,

@@ -168,6 +168,41 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
                     loss_dev, ws, ws_bytes);
 }
 
+kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,
+                            int64_t K, float alpha, const float *A, int64_t lda,
+                            int a_mn, const float *B, int64_t ldb, int b_mn,
+                            float beta, float *C, int64_t ldc, int32_t *info_dev) {
+  if (M < 0 || N < 0 || K < 0 || !info_dev) return KRONQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return KRONQ_OK;
+  if (!C || (K > 0 && (!A || !B))) return KRONQ_ERR_INVALID_ARG;
+  const int64_t a_rows = a_mn ? K : M, a_cols = a_mn ? M : K;
+  const int64_t b_rows = b_mn ? K : N, b_cols = b_mn ? N : K;
+  if (ldc < N || (K > 0 && (lda < a_cols || ldb < b_cols))) return KRONQ_ERR_INVALID_ARG;
+  if (!aligned(C, 16) || ldc % 4 || (K > 0 && (!aligned(A, 16) || !aligned(B, 16) ||
+                                                lda % 4 || ldb % 4)))
+    return KRONQ_ERR_UNSUPPORTED;
+  if (K > 0) {
+    auto overlap = [](const float *p, int64_t rows, int64_t ld, int64_t cols,
+                      const float *q, int64_t qrows, int64_t qld, int64_t qcols) {
+      const float *pe = p + (rows - 1) * ld + cols, *qe = q + (qrows - 1) * qld + qcols;
+      return p < qe && q < pe;
+    };
+    if (overlap(C, M, ldc, N, A, a_rows, lda, a_cols) ||
+        overlap(C, M, ldc, N, B, b_rows, ldb, b_cols))
+      return KRONQ_ERR_INVALID_ARG;
+  }
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  GemmArgs g;
+  g.M = M; g.N = N; g.K = K;
+  g.A = A; g.lda = lda; g.a_mn = a_mn != 0;
+  g.B = B; g.ldb = ldb; g.b_mn = b_mn != 0;
+  g.C = C; g.ldc = ldc;
+  g.alpha = alpha; g.beta = beta;
+  return gemm_tf32x3(st, g, info_dev);
+}
+
 kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,
                                  int n, double avg_budget, int *bits_out) {
   if (!score || !numel || !bits_out || n <= 0 || !(avg_budget >= 2.0))

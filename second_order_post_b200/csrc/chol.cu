@@ -225,13 +225,6 @@ __global__ void __launch_bounds__(LTHREADS)
   }
 }
 
-__global__ void zero_lower_kernel(float *H, int64_t d) {
-  const int64_t r = blockIdx.y;
-  for (int64_t c = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; c < r;
-       c += int64_t(gridDim.x) * blockDim.x)
-    H[r * d + c] = 0.f;
-}
-
 constexpr int MAXD = 40;  // recursion depth bound (d <= 65536 gives <= 10)
 
 struct Ctx {
@@ -349,36 +342,49 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.kflags = KR_A_UPPER;
     KQ_TRY(gemm_tf32x3(c.st, g, c.info));
   }
+  // zeros below the diagonal of this node (the leaves zero their own blocks):
+  // triangular operands of the parents' products read U as 128 x 256 tiles
+  if (cudaMemset2DAsync(c.H + (off + h) * d + off, static_cast<size_t>(d) * 4, 0,
+                        static_cast<size_t>(h) * 4, static_cast<size_t>(m),
+                        c.st) != cudaSuccess)
+    return KRONQ_ERR_CUDA;
   return KRONQ_OK;
 }
 
-// Workspace layout: [V slot, T slot] per recursion depth, then lambda. The
+// Workspace layout: [V, T] slots per recursion depth, then lambda. The
 // largest node at depth i+1 is the larger child m_i of the largest node at i.
-size_t chol_layout(int64_t d, size_t *v_off, size_t *t_off, int *depths) {
+struct CholLayout {
+  size_t v[MAXD], t[MAXD];
+  int depths;
+  size_t total;
+};
+CholLayout chol_layout(int64_t d) {
   auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  CholLayout L{};
   size_t off = 0;
   int k = 0;
   for (int64_t n = d; n > NB && k < MAXD; ++k) {
     const int64_t h = first_half(n);
     const size_t slot = al(static_cast<size_t>(h) * (n - h) * 4);
-    if (v_off) v_off[k] = off;
-    if (t_off) t_off[k] = off + slot;
+    L.v[k] = off;
+    L.t[k] = off + slot;
     off += 2 * slot;
     n = n - h;
   }
-  if (depths) *depths = k;
-  return off + 256;
+  L.depths = k;
+  L.total = off + 256;
+  return L;
 }
 
 }  // namespace
 
-size_t chol_ws_bytes(int64_t d) { return chol_layout(d, nullptr, nullptr, nullptr); }
+size_t chol_ws_bytes(int64_t d) { return chol_layout(d).total; }
 
 kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
                       void *ws, size_t ws_bytes, int32_t *info) {
-  size_t v_off[MAXD], t_off[MAXD];
-  int depths = 0;
-  const size_t need = chol_layout(d, v_off, t_off, &depths);
+  const CholLayout lay = chol_layout(d);
+  const int depths = lay.depths;
+  const size_t need = lay.total;
   if (ws_bytes < need) return KRONQ_ERR_INVALID_ARG;
   CholStreams *cs = nullptr;
   KQ_TRY(chol_streams(&cs));
@@ -387,12 +393,15 @@ kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
   c.st = cs->main;
   c.H = H;
   c.d = d;
+  auto at = [&](int k, size_t o) {
+    return k < depths ? reinterpret_cast<float *>(w + o) : nullptr;
+  };
   for (int k = 0; k < MAXD; ++k) {
     c.side[k] = cs->side[k];
     c.ev_v[k] = cs->ev_v[k];
     c.ev_t[k] = cs->ev_t[k];
-    c.V[k] = k < depths ? reinterpret_cast<float *>(w + v_off[k]) : nullptr;
-    c.T[k] = k < depths ? reinterpret_cast<float *>(w + t_off[k]) : nullptr;
+    c.V[k] = at(k, lay.v[k]);
+    c.T[k] = at(k, lay.t[k]);
   }
   float *lambda = reinterpret_cast<float *>(w + need - 256);
   c.lambda = lambda;
@@ -406,10 +415,6 @@ kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
   damping_kernel<<<1, 1024, 0, c.st>>>(H, d, damp_rel, lambda, info);
   KQ_CHECK_LAUNCH();
   KQ_TRY(rinv(c, 0, d, 0));
-  dim3 grid(static_cast<unsigned>(kq_min<int64_t>(ceil_div(d, 256), 64)),
-            static_cast<unsigned>(d));
-  zero_lower_kernel<<<grid, 256, 0, c.st>>>(H, d);
-  KQ_CHECK_LAUNCH();
   // join back into the caller's stream (every side stream is idle by now
   // from the main stream's point of view; joining them keeps ws reuse safe)
   if (cudaEventRecord(cs->join_main, cs->main) != cudaSuccess ||

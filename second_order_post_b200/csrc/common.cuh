@@ -38,12 +38,14 @@ kronq_status require_sm100();
 
 // 2D tiled tensor map over a row-major fp32/bf16 matrix: inner extent `inner`
 // (contiguous), outer extent `outer`, row pitch `pitch_elems`, box
-// {box_inner, box_outer}, 128-byte swizzle (16-byte granules, or 32-byte
-// granules with swz32), zero fill out of bounds.
+// {box_inner, box_outer}, zero fill out of bounds. Swizzle: TMAP_SW128
+// (128-byte rows, 16-byte granules), TMAP_SW128_32B (128-byte rows, 32-byte
+// granules) or TMAP_SW64 (64-byte rows, 16-byte granules).
+enum { TMAP_SW128 = 0, TMAP_SW128_32B = 1, TMAP_SW64 = 2 };
 kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
                           uint64_t inner, uint64_t outer, uint64_t pitch_elems,
                           uint32_t box_inner, uint32_t box_outer,
-                          bool swz32 = false);
+                          int swz = TMAP_SW128);
 
 inline cudaStream_t as_stream(kronq_stream_t s) {
   return reinterpret_cast<cudaStream_t>(s);
@@ -105,15 +107,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but the thread may sleep in hardware until the phase completes
+// or about `ns` nanoseconds pass (no polling traffic on shared memory).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete. Returns
 // false (and leaves the barrier untouched) once *abort is set by another
-// thread or the wall-time limit passes; the caller then winds down.
+// thread or the wall-time limit passes; the caller then winds down. Between
+// checks the thread sleeps on the barrier for up to 0.5 ms.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
       *abort = 1;
@@ -218,9 +236,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 
 // Shared-memory matrix descriptor for tcgen05 (version field 1; offsets in
 // bytes). Layout type 2 = 128-byte swizzle with 16-byte granules (K-major
-// operands, and MN-major 16-bit operands); layout type 1 = 128-byte swizzle
-// with 32-byte granules, the only MN-major layout for 32-bit (tf32) operands
-// (K groups of 4 rows instead of 8).
+// operands, and MN-major 16-bit operands); layout type 4 = the same with
+// 64-byte rows; layout type 1 = 128-byte swizzle with 32-byte granules, the
+// only MN-major layout for 32-bit (tf32) operands (K groups of 4 rows
+// instead of 8).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo,
                                           uint32_t sbo, uint32_t layout) {
   uint64_t d = 0;
@@ -243,6 +262,21 @@ __host__ __device__ constexpr uint32_t idesc_make(uint32_t fmt, uint32_t a_mn,
                                                   uint32_t N) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) |
          ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// The tf32 MMA reads an fp32 operand by dropping its 13 low mantissa bits
+// (truncation, measured on sm_100a), so the raw slab already is the hi part;
+// only lo = x - trunc(x) (exact in fp32, |lo| < 2^-10 |x|) has to be written.
+// lo is stored rounded to the nearest tf32 value, so the MMA's own truncation
+// of it costs nothing; per product the split then keeps a*b up to
+// |a_lo b_lo| + 2^-22 (|a| |b_lo| + |a_lo| |b|) <= 1.5 * 2^-20 |a b|.
+__device__ __forceinline__ float tf32_lo1(float x) {
+  const float lo = x - __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+  // nearest tf32 value, ties away from zero (sign-magnitude bit pattern)
+  return __uint_as_float((__float_as_uint(lo) + 0x1000u) & 0xffffe000u);
+}
+__device__ __forceinline__ float4 tf32_lo(float4 x) {
+  return make_float4(tf32_lo1(x.x), tf32_lo1(x.y), tf32_lo1(x.z), tf32_lo1(x.w));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

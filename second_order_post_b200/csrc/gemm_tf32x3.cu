@@ -3,23 +3,27 @@
 // MMAs (hi*hi + hi*lo + lo*hi) per k-step into an fp32 TMEM accumulator.
 //
 // Used by the blocked Cholesky/inverse, the OBS trailing updates and the
-// layer loss. One CTA computes a 128x128 tile:
-//   warp 0      TMA producer (one elected lane), 3-stage ring of 32-wide k-slabs
+// layer loss. One CTA computes a 128 x BN tile (BN = 256 for wide outputs,
+// 128 otherwise):
+//   warp 0      TMA producer (one elected lane), ring of BK-wide k-slabs
 //   warp 1      TMEM owner and MMA issuer (one elected lane)
 //   warps 2..5  write the TF32 low part of each landed fp32 slab next to it in
 //               shared memory (the raw slab itself serves as the high part),
 //               then run the epilogue (TMEM -> registers -> C).
+// The split warps load a whole slab into registers before they store any low
+// part (the two share one array, so interleaved loads and stores would run
+// one round trip at a time). Low parts precomputed in global memory instead
+// would double the L2 -> SM traffic, which costs more than the split.
 #include "kernels.cuh"
 
 namespace kronq {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 32, STAGES = 3;
-constexpr int TILE_BYTES = BM * BK * 4;        // one 128 x 32 fp32 slab
-constexpr int STAGE_BYTES = 4 * TILE_BYTES;    // A_hi, A_lo, B_hi, B_lo
+constexpr int BM = 128;
 constexpr int NTHREADS = 192;
 constexpr int GROUP_M = 16;                    // tile raster: 16 rows per band
 
+template <int STAGES>
 struct Ctl {
   uint64_t full[STAGES];   // TMA landed (expect_tx)
   uint64_t conv[STAGES];   // hi/lo split written (128 arrivals)
@@ -29,43 +33,71 @@ struct Ctl {
   uint32_t tmem_base;
   int abort;
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + sizeof(Ctl) + 64;
 
-// The tf32 MMA reads an fp32 operand by dropping its 13 low mantissa bits
-// (truncation, measured on sm_100a), so the raw slab already is the hi part;
-// only lo = x - trunc(x) (exact in fp32) has to be written.
-__device__ __forceinline__ float4 tf32_lo(float4 x) {
-  const uint32_t mask = 0xffffe000u;
-  return make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & mask),
-                     x.y - __uint_as_float(__float_as_uint(x.y) & mask),
-                     x.z - __uint_as_float(__float_as_uint(x.z) & mask),
-                     x.w - __uint_as_float(__float_as_uint(x.w) & mask));
+// Tile configuration: BN output columns, BK-wide k-slabs, STAGES-deep ring.
+// K-major slabs are rows of BK fp32 (128 or 64 bytes, swizzled to match);
+// MN-major slabs are 32-wide MN chunks of BK k-rows (32-byte granules).
+template <int BN_, int BK_, int STAGES_>
+struct Cfg {
+  static constexpr int BN = BN_, BK = BK_, STAGES = STAGES_;
+  static constexpr int TA = BM * BK * 4;           // one A slab (bytes)
+  static constexpr int TB = BN * BK * 4;           // one B slab
+  static constexpr int STAGE = 2 * TA + 2 * TB;    // A_hi, A_lo, B_hi, B_lo
+  static constexpr int SMEM = STAGES * STAGE + 1024 + sizeof(Ctl<STAGES>) + 64;
+  static constexpr uint32_t K_LAYOUT = BK * 4 == 128 ? 2 : 4;  // SW128 / SW64
+  static constexpr int K_TMAP = BK * 4 == 128 ? TMAP_SW128 : TMAP_SW64;
+  static constexpr uint32_t K_SBO = 8 * BK * 4;    // 8-row group
+  static constexpr uint32_t MN_CHUNK = BK * 128;   // one 32-wide MN chunk
+  static_assert(BK * 4 == 128 || BK * 4 == 64, "k-slab rows of 64 or 128 bytes");
+  static_assert(BN == 128 || BN == 256, "tile width");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+using Narrow = Cfg<128, 32, 3>;
+using Wide = Cfg<256, 16, 4>;
+
+// First column tile on or right of the diagonal for row tile bi.
+template <class C>
+__host__ __device__ constexpr int64_t upper_first(int64_t bi) {
+  return bi * BM / C::BN;
 }
 
+struct GemmP {
+  int64_t M, N, K;
+  float *C;
+  int64_t ldc;
+  float alpha, beta;
+  uint32_t kflags;
+  int a_mn, b_mn, upper_only, tiles_m, tiles_n, vec_ok;
+  int32_t *info;
+};
+
+template <class C>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA,
-                       const __grid_constant__ CUtensorMap tmB, int64_t M,
-                       int64_t N, int64_t K, float *__restrict__ C, int64_t ldc,
-                       float alpha, float beta, uint32_t kflags, int a_mn,
-                       int b_mn, int upper_only, int tiles_m, int tiles_n,
-                       int vec_ok, int32_t *info) {
+                       const __grid_constant__ CUtensorMap tmB, const GemmP p) {
+  constexpr int BN = C::BN, BK = C::BK, STAGES = C::STAGES;
+  constexpr int TA = C::TA, TB = C::TB;
+  const int64_t M = p.M, N = p.N, K = p.K;
+  const int a_mn = p.a_mn, b_mn = p.b_mn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctl *ctl = reinterpret_cast<Ctl *>(smem + STAGES * STAGE_BYTES);
+  Ctl<STAGES> *ctl = reinterpret_cast<Ctl<STAGES> *>(smem + STAGES * C::STAGE);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_n = p.tiles_n, tiles_m = p.tiles_m;
+  const uint32_t kflags = p.kflags;
 
   // ---- tile coordinates
   int64_t bi, bj;
   {
     int64_t t = blockIdx.x;
-    if (upper_only) {
+    if (p.upper_only) {
       bi = 0;
-      while (t >= tiles_n - bi) {
-        t -= tiles_n - bi;
+      while (t >= tiles_n - upper_first<C>(bi)) {
+        t -= tiles_n - upper_first<C>(bi);
         ++bi;
       }
-      bj = bi + t;
+      bj = upper_first<C>(bi) + t;
     } else {
       const int64_t band = t / (int64_t(GROUP_M) * tiles_n);
       const int64_t rows = kq_min<int64_t>(GROUP_M, tiles_m - band * GROUP_M);
@@ -98,7 +130,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, 128);
+    tmem_alloc(&ctl->tmem_base, BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -115,22 +147,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (it >= STAGES &&
             !mbar_wait(&ctl->empty[s], ((it / STAGES) - 1) & 1, abort))
           break;
-        uint8_t *st = smem + s * STAGE_BYTES;
+        uint8_t *st = smem + s * C::STAGE;
         const int32_t k0 = static_cast<int32_t>(kb + int64_t(it) * BK);
-        mbar_expect_tx(&ctl->full[s], 2 * TILE_BYTES);
+        mbar_expect_tx(&ctl->full[s], TA + TB);
         if (!a_mn) {
           tma_load_2d(st, &tmA, &ctl->full[s], k0, static_cast<int32_t>(m0));
         } else {
-          for (int c = 0; c < 4; ++c)
-            tma_load_2d(st + c * (TILE_BYTES / 4), &tmA, &ctl->full[s],
+          for (int c = 0; c < BM / 32; ++c)
+            tma_load_2d(st + c * C::MN_CHUNK, &tmA, &ctl->full[s],
                         static_cast<int32_t>(m0 + 32 * c), k0);
         }
-        uint8_t *sb = st + 2 * TILE_BYTES;
+        uint8_t *sb = st + 2 * TA;
         if (!b_mn) {
           tma_load_2d(sb, &tmB, &ctl->full[s], k0, static_cast<int32_t>(n0));
         } else {
-          for (int c = 0; c < 4; ++c)
-            tma_load_2d(sb + c * (TILE_BYTES / 4), &tmB, &ctl->full[s],
+          for (int c = 0; c < BN / 32; ++c)
+            tma_load_2d(sb + c * C::MN_CHUNK, &tmB, &ctl->full[s],
                         static_cast<int32_t>(n0 + 32 * c), k0);
         }
         issued = it + 1;
@@ -139,21 +171,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_make(2, a_mn, b_mn, BM, BN);
-      const uint32_t lbo_a = a_mn ? TILE_BYTES / 4 : 16;
-      const uint32_t lbo_b = b_mn ? TILE_BYTES / 4 : 16;
-      // K-major: 8-row groups of 128 B rows (16-byte swizzle granules);
+      // K-major: 8-row groups of BK-float rows (16-byte swizzle granules);
       // MN-major tf32: 4-row groups, 32-byte granules (layout type 1)
-      const uint32_t sbo_a = a_mn ? 512 : 1024, sbo_b = b_mn ? 512 : 1024;
-      const uint32_t lay_a = a_mn ? 1 : 2, lay_b = b_mn ? 1 : 2;
+      const uint32_t lbo_a = a_mn ? C::MN_CHUNK : 16;
+      const uint32_t lbo_b = b_mn ? C::MN_CHUNK : 16;
+      const uint32_t sbo_a = a_mn ? 512 : C::K_SBO, sbo_b = b_mn ? 512 : C::K_SBO;
+      const uint32_t lay_a = a_mn ? 1 : C::K_LAYOUT, lay_b = b_mn ? 1 : C::K_LAYOUT;
       int it = 0;
       for (; it < nk; ++it) {
         const int s = it % STAGES;
         if (!mbar_wait(&ctl->conv[s], (it / STAGES) & 1, abort)) break;
         tc_fence_after();
-        const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
-        const uint32_t a_lo = a_hi + TILE_BYTES;
-        const uint32_t b_hi = a_hi + 2 * TILE_BYTES;
-        const uint32_t b_lo = a_hi + 3 * TILE_BYTES;
+        const uint32_t a_hi = smem_u32(smem + s * C::STAGE);
+        const uint32_t a_lo = a_hi + TA;
+        const uint32_t b_hi = a_hi + 2 * TA;
+        const uint32_t b_lo = b_hi + TB;
 #pragma unroll
         for (int kk = 0; kk < BK / 8; ++kk) {
           const uint32_t ao = a_mn ? kk * 1024 : kk * 32;
@@ -179,13 +211,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int it = 0; it < nk; ++it) {
       const int s = it % STAGES;
       if (!mbar_wait(&ctl->full[s], (it / STAGES) & 1, abort)) break;
-      float4 *st = reinterpret_cast<float4 *>(smem + s * STAGE_BYTES);
-      constexpr int Q = TILE_BYTES / 16;
-#pragma unroll 4
-      for (int i = ct; i < Q; i += 128) {
-        st[Q + i] = tf32_lo(st[i]);
-        st[3 * Q + i] = tf32_lo(st[2 * Q + i]);
-      }
+      float4 *sa = reinterpret_cast<float4 *>(smem + s * C::STAGE);
+      float4 *sb = sa + 2 * (TA / 16);
+      // all loads first: the slabs and their low parts share one array
+      float4 ra[TA / 16 / 128], rb[TB / 16 / 128];
+#pragma unroll
+      for (int j = 0; j < TA / 16 / 128; ++j) ra[j] = sa[ct + 128 * j];
+#pragma unroll
+      for (int j = 0; j < TB / 16 / 128; ++j) rb[j] = sb[ct + 128 * j];
+#pragma unroll
+      for (int j = 0; j < TA / 16 / 128; ++j) sa[TA / 16 + ct + 128 * j] = tf32_lo(ra[j]);
+#pragma unroll
+      for (int j = 0; j < TB / 16 / 128; ++j) sb[TB / 16 + ct + 128 * j] = tf32_lo(rb[j]);
       fence_proxy_async_smem();
       mbar_arrive(&ctl->conv[s]);
     }
@@ -196,6 +233,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q = warp & 3;
     const int64_t row = m0 + 32 * q + lane;
     for (int c = 0; c < BN / 32; ++c) {
+      const int64_t col0 = n0 + 32 * c;
+      if (col0 >= N) break;
       float v[32];
       if (have) {
         tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 32 * c, v);
@@ -204,27 +243,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int t = 0; t < 32; ++t) v[t] = 0.f;
       }
       if (row >= M) continue;
-      const int64_t col0 = n0 + 32 * c;
-      float *crow = C + row * ldc + col0;
-      if (vec_ok && col0 + 32 <= N) {
+      float *crow = p.C + row * p.ldc + col0;
+      if (p.vec_ok && col0 + 32 <= N) {
 #pragma unroll
         for (int t = 0; t < 32; t += 4) {
-          float4 o = make_float4(alpha * v[t], alpha * v[t + 1],
-                                 alpha * v[t + 2], alpha * v[t + 3]);
-          if (beta != 0.f) {
+          float4 o = make_float4(p.alpha * v[t], p.alpha * v[t + 1],
+                                 p.alpha * v[t + 2], p.alpha * v[t + 3]);
+          if (p.beta != 0.f) {
             const float4 old = *reinterpret_cast<const float4 *>(crow + t);
-            o.x += beta * old.x;
-            o.y += beta * old.y;
-            o.z += beta * old.z;
-            o.w += beta * old.w;
+            o.x += p.beta * old.x;
+            o.y += p.beta * old.y;
+            o.z += p.beta * old.z;
+            o.w += p.beta * old.w;
           }
           *reinterpret_cast<float4 *>(crow + t) = o;
         }
       } else {
-        for (int t = 0; t < 32 && col0 + t < N; ++t) {
-          float o = alpha * v[t];
-          if (beta != 0.f) o += beta * crow[t];
-          crow[t] = o;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if (col0 + t < N) {
+            float o = p.alpha * v[t];
+            if (p.beta != 0.f) o += p.beta * crow[t];
+            crow[t] = o;
+          }
         }
       }
     }
@@ -234,7 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (ctl->abort) {
-    if (threadIdx.x == 0) report(info, KRONQ_ERR_TIMEOUT);
+    if (threadIdx.x == 0) report(p.info, KRONQ_ERR_TIMEOUT);
     if (warp == 0 && lane == 0) {
       const uint64_t t0 = globaltimer();
       for (int s = 0; s < STAGES && s < issued; ++s) {
@@ -254,8 +295,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 128);
+    tmem_dealloc(tbase, BN);
   }
+}
+
+template <class C>
+kronq_status launch(cudaStream_t st, const GemmArgs &g, int32_t *info) {
+  CUtensorMap ta, tb;
+  // A: K-major -> rows M of K; MN-major -> rows K of M (32-wide chunks)
+  if (g.K > 0) {
+    KQ_TRY(g.a_mn ? make_tmap_2d(&ta, g.A, false, g.M, g.K, g.lda, 32, C::BK, TMAP_SW128_32B)
+                  : make_tmap_2d(&ta, g.A, false, g.K, g.M, g.lda, C::BK, BM, C::K_TMAP));
+    KQ_TRY(g.b_mn ? make_tmap_2d(&tb, g.B, false, g.N, g.K, g.ldb, 32, C::BK, TMAP_SW128_32B)
+                  : make_tmap_2d(&tb, g.B, false, g.K, g.N, g.ldb, C::BK, C::BN, C::K_TMAP));
+  } else {
+    memset(&ta, 0, sizeof(ta));
+    memset(&tb, 0, sizeof(tb));
+  }
+  const int64_t tm = ceil_div(g.M, BM), tn = ceil_div(g.N, C::BN);
+  int64_t tiles = tm * tn;
+  if (g.upper_tiles_only) {
+    tiles = 0;
+    for (int64_t bi = 0; bi < tm; ++bi) tiles += tn - upper_first<C>(bi);
+  }
+  if (tiles > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(gemm_tf32x3_kernel<C>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+    attr_done = true;
+  }
+  GemmP p;
+  p.M = g.M; p.N = g.N; p.K = g.K;
+  p.C = g.C; p.ldc = g.ldc;
+  p.alpha = g.alpha; p.beta = g.beta;
+  p.kflags = g.kflags;
+  p.a_mn = g.a_mn ? 1 : 0;
+  p.b_mn = g.b_mn ? 1 : 0;
+  p.upper_only = g.upper_tiles_only ? 1 : 0;
+  p.tiles_m = static_cast<int>(tm);
+  p.tiles_n = static_cast<int>(tn);
+  p.vec_ok = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc % 4 == 0);
+  p.info = info;
+  gemm_tf32x3_kernel<C><<<static_cast<unsigned>(tiles), NTHREADS, C::SMEM, st>>>(
+      ta, tb, p);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
 }
 
 }  // namespace
@@ -264,35 +351,13 @@ kronq_status gemm_tf32x3(cudaStream_t st, const GemmArgs &g, int32_t *info) {
   if (g.M < 0 || g.N < 0 || g.K < 0) return KRONQ_ERR_INVALID_ARG;
   if (g.M == 0 || g.N == 0) return KRONQ_OK;
   if (g.upper_tiles_only && g.M != g.N) return KRONQ_ERR_INVALID_ARG;
-  CUtensorMap ta, tb;
-  // A: K-major -> rows M of K; MN-major -> rows K of M
-  if (g.K > 0) {
-    KQ_TRY(make_tmap_2d(&ta, g.A, false, g.a_mn ? g.M : g.K,
-                        g.a_mn ? g.K : g.M, g.lda, 32, g.a_mn ? 32 : 128, g.a_mn));
-    KQ_TRY(make_tmap_2d(&tb, g.B, false, g.b_mn ? g.N : g.K,
-                        g.b_mn ? g.K : g.N, g.ldb, 32, g.b_mn ? 32 : 128, g.b_mn));
-  } else {
-    memset(&ta, 0, sizeof(ta));
-    memset(&tb, 0, sizeof(tb));
-  }
-  const int64_t tm = ceil_div(g.M, BM), tn = ceil_div(g.N, BN);
-  const int64_t tiles = g.upper_tiles_only ? tn * (tn + 1) / 2 : tm * tn;
-  if (tiles > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(gemm_tf32x3_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr_done = true;
-  }
-  const int vec_ok = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc % 4 == 0);
-  gemm_tf32x3_kernel<<<static_cast<unsigned>(tiles), NTHREADS, SMEM_BYTES, st>>>(
-      ta, tb, g.M, g.N, g.K, g.C, g.ldc, g.alpha, g.beta, g.kflags,
-      g.a_mn ? 1 : 0, g.b_mn ? 1 : 0, g.upper_tiles_only ? 1 : 0,
-      static_cast<int>(tm), static_cast<int>(tn), vec_ok, info);
-  KQ_CHECK_LAUNCH();
-  return KRONQ_OK;
+  // wide tiles when they fill the GPU at least once and waste at most an
+  // eighth of the last column tile's width
+  const int64_t wide_tiles = ceil_div(g.M, BM) * ceil_div(g.N, Wide::BN);
+  const int64_t pad = ceil_div(g.N, Wide::BN) * Wide::BN - g.N;
+  if (wide_tiles >= 148 && pad * 8 <= ceil_div(g.N, Wide::BN) * Wide::BN)
+    return launch<Wide>(st, g, info);
+  return launch<Narrow>(st, g, info);
 }
 
 }  // namespace kronq

@@ -79,7 +79,7 @@ kronq_status require_sm100() {
 kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
                           uint64_t inner, uint64_t outer, uint64_t pitch_elems,
                           uint32_t box_inner, uint32_t box_outer,
-                          bool swz32) {
+                          int swz) {
   const uint64_t es = bf16 ? 2 : 4;
   if (reinterpret_cast<uintptr_t>(base) % 16 != 0) return KRONQ_ERR_UNSUPPORTED;
   if ((pitch_elems * es) % 16 != 0) return KRONQ_ERR_UNSUPPORTED;
@@ -93,7 +93,9 @@ kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
                   bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                   2, const_cast<void *>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swz32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                  swz == TMAP_SW128_32B ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                  : swz == TMAP_SW64    ? CU_TENSOR_MAP_SWIZZLE_64B
+                                        : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? KRONQ_OK : KRONQ_ERR_CUDA;

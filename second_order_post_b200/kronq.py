@@ -78,6 +78,8 @@ _SIGS = {
     "kronq_quantize_sublayer": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p,
                                 _sz, _p],
     "kronq_layer_loss": [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _sz],
+    "kronq_gemm_f32": [_p, _i64, _i64, _i64, _f, _p, _i64, ctypes.c_int, _p,
+                       _i64, ctypes.c_int, _f, _p, _i64, _p],
     "kronq_workspace_bytes": [ctypes.c_int, _i64, _i64, _OPTS],
     "kronq_allocate_bits": [_p, _p, ctypes.c_int, _d, _p],
     "kronq_status_string": [ctypes.c_int],
@@ -174,6 +176,17 @@ def kronq_layer_loss(W_ref, W_hat, H_X, H_G, loss, ws, stream=None):
     _check("kronq_layer_loss", _lib.kronq_layer_loss(
         _stream(stream), _ptr(W_ref), _ptr(W_hat), _ptr(H_X), _ptr(H_G), d_out,
         d_in, _ptr(loss), _ptr(ws), ws.numel() * ws.element_size()))
+
+
+def kronq_gemm_f32(A, B, C, info, alpha=1.0, beta=0.0, a_mn=False, b_mn=False,
+                   stream=None):
+    """C = alpha * A Bᵀ + beta * C; A is M x K (or K x M with a_mn), B is
+    N x K (or K x N with b_mn); all 2-D fp32 CUDA tensors, rows contiguous."""
+    M, N = C.shape
+    K = A.shape[0] if a_mn else A.shape[1]
+    _check("kronq_gemm_f32", _lib.kronq_gemm_f32(
+        _stream(stream), M, N, K, alpha, _ptr(A), A.stride(0), int(a_mn),
+        _ptr(B), B.stride(0), int(b_mn), beta, _ptr(C), C.stride(0), _ptr(info)))
 
 
 def kronq_allocate_bits(scores, numel, avg_budget):

@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "kronq.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(kronq_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(kronq_[a-z0-9_]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -63,6 +63,15 @@ def test_invalid_args_rejected_before_device(K):
                           1 << 20, p) == K.KRONQ_ERR_UNSUPPORTED
     assert lib.kronq_chol_inv(None, p, 100, 0.01, p, 1 << 20, p) == K.KRONQ_ERR_UNSUPPORTED
     assert lib.kronq_chol_inv(None, p, 128, -1.0, p, 1 << 20, p) == K.KRONQ_ERR_INVALID_ARG
+    # gemm: negative sizes, short pitches, misalignment, C overlapping A
+    g = lib.kronq_gemm_f32
+    q = ctypes.c_void_p(1 << 20)
+    assert g(None, -1, 8, 8, 1.0, p, 8, 0, p, 8, 0, 0.0, q, 8, p) == K.KRONQ_ERR_INVALID_ARG
+    assert g(None, 8, 8, 8, 1.0, p, 4, 0, p, 8, 0, 0.0, q, 8, p) == K.KRONQ_ERR_INVALID_ARG
+    assert g(None, 8, 8, 8, 1.0, ctypes.c_void_p(260), 8, 0, p, 8, 0, 0.0, q, 8,
+             p) == K.KRONQ_ERR_UNSUPPORTED
+    assert g(None, 8, 8, 8, 1.0, p, 8, 0, q, 8, 0, 0.0, p, 8, p) == K.KRONQ_ERR_INVALID_ARG
+    assert g(None, 0, 8, 8, 1.0, nullp, 8, 0, nullp, 8, 0, 0.0, nullp, 8, p) == K.KRONQ_OK
 
 
 def test_workspace_sizes(K):

@@ -136,7 +136,9 @@ def test_biip(cuda_device, case):
 
 
 # ------------------------------------------------------------------ Cholesky
-@pytest.mark.parametrize("d", [128, 256, 512, 640, 1024])
+# 6016 = 47 blocks of 128: a ragged split whose products (SYRK included) run
+# on the 128 x 256 GEMM tiles
+@pytest.mark.parametrize("d", [128, 256, 512, 640, 1024, 6016])
 def test_chol_inv(cuda_device, d):
     Kq = K()
     h = synth.make_spd(d, seed=d, cond_spread=2.0)
@@ -235,10 +237,76 @@ def test_quantize(cuda_device, d_out, d_in, bits, group):
     assert rel_fro(f64(W), rep["w_hat"]) < 1e-5
 
 
-# ------------------------------------------------------------------ loss
-def test_layer_loss(cuda_device):
+def test_quantize_sampled_rows(cuda_device):
+    """A layer large enough for the 128 x 256 GEMM tiles in the trailing
+    updates; rows are independent given U, so the oracle checks a sample."""
     Kq = K()
-    d_out, d_in = 256, 384
+    d_out, d_in, bits, group = 2048, 4096, 2, 128
+    data = synth.small_case(d_out, d_in, 2 * d_in, seed=11)
+    w32 = data["W"].numpy().astype(np.float32)
+    u32 = O.chol_inv(O.cov(data["X"].numpy()), 0.01).astype(np.float32)
+    opts = Kq.make_opts(bits=bits, group=group)
+    W = dev(w32)
+    codes = torch.empty(d_out, bits * d_in // 32, dtype=torch.int32, device="cuda")
+    scales = torch.empty(d_out, d_in // group, device="cuda")
+    zeros = torch.empty(d_out, d_in // group, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(Kq.kronq_workspace_bytes(Kq.KRONQ_WS_QUANT, d_out, d_in, opts),
+                     dtype=torch.uint8, device="cuda")
+    info = torch.ones(1, dtype=torch.int32, device="cuda")
+    Kq.kronq_quantize_sublayer(opts, W, dev(u32), codes, scales, zeros, ws, info)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    rows = np.random.default_rng(0).choice(d_out, 48, replace=False)
+    got_codes = O.unpack_codes(codes.cpu().numpy().view(np.uint32), bits, d_in)[rows]
+    got_zeros = zeros.cpu().numpy().astype(np.int64)[rows]
+    w64, u64 = w32[rows].astype(np.float64), u32.astype(np.float64)
+    ident, n_bad, _ = replay_check(w64, u64, got_codes, got_zeros, bits, group)
+    assert n_bad == 0
+    assert ident >= 0.999
+
+
+# ------------------------------------------------------------------ GEMM
+# (M, N, K, a_mn, b_mn): narrow 128 x 128 tiles, ragged edges, and the wide
+# 128 x 256 tiles in every operand major
+GEMM_CASES = [(300, 200, 100, 0, 0), (256, 384, 1000, 1, 0), (129, 132, 64, 0, 1),
+              (2048, 4096, 4096, 0, 0), (2048, 4096, 1536, 1, 1),
+              (1920, 3968, 2080, 0, 1), (4096, 2816, 512, 1, 0)]
+
+
+@pytest.mark.parametrize("case", GEMM_CASES)
+def test_gemm_f32(cuda_device, case):
+    """Elementwise against fp64. Each product keeps all but
+    1.5 * 2^-20 |a b| (truncated hi, rounded lo, no lo*lo term) and the
+    3K/8 fp32 accumulation steps add rounding that grows like their square
+    root: |err| <= (1.5 * 2^-20 + 2 sqrt(3K) 2^-24) |alpha| (|A| |B|^T)
+    plus one rounding of the result. A missing or misplaced hi/lo term
+    costs ~2^-11 per product and fails this by two orders of magnitude."""
+    Kq = K()
+    M, N, Kd, a_mn, b_mn = case
+    g = torch.Generator(device="cuda").manual_seed(M + N + Kd)
+    a = torch.randn(M, Kd, device="cuda", generator=g) * torch.exp(
+        torch.randn(1, Kd, device="cuda", generator=g))
+    b = torch.randn(N, Kd, device="cuda", generator=g)
+    c0 = torch.randn(M, N, device="cuda", generator=g)
+    A = a.T.contiguous() if a_mn else a
+    B = b.T.contiguous() if b_mn else b
+    C = c0.clone()
+    info = torch.ones(1, dtype=torch.int32, device="cuda")
+    Kq.kronq_gemm_f32(A, B, C, info, alpha=-0.5, beta=2.0, a_mn=a_mn, b_mn=b_mn)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    want = 2.0 * c0.double() - 0.5 * (a.double() @ b.double().T)
+    rel = 1.5 * 2.0 ** -20 + 2 * math.sqrt(3 * Kd) * 2.0 ** -24
+    bound = rel * 0.5 * (a.double().abs() @ b.double().abs().T) + \
+        2.0 ** -23 * want.abs() + 1e-30
+    err = (C.double() - want).abs()
+    assert bool((err <= bound).all()), float((err / bound).max())
+
+
+# ------------------------------------------------------------------ loss
+@pytest.mark.parametrize("d_out,d_in", [(256, 384), (2048, 4096)])
+def test_layer_loss(cuda_device, d_out, d_in):
+    Kq = K()
     rng = np.random.default_rng(3)
     a = rng.standard_normal((d_out, d_in)).astype(np.float32)
     b = (a + 0.01 * rng.standard_normal((d_out, d_in))).astype(np.float32)
@@ -250,4 +318,13 @@ def test_layer_loss(cuda_device):
     Kq.kronq_layer_loss(dev(a), dev(b), hx.cuda(), hg.cuda(), loss, ws)
     torch.cuda.synchronize()
     want = O.layer_loss(a.astype(np.float64) - b, hx.double().numpy(), hg.double().numpy())
-    assert math.isclose(loss.item(), want, rel_tol=1e-5)
+    # error budget of the two fp32-accurate products P = D H_X, Q = H_G D
+    # (per element as in test_gemm_f32) carried through sum(P * Q)
+    dd = torch.from_numpy(a.astype(np.float64) - b).cuda()
+    hxd, hgd = hx.double().cuda(), hg.double().cuda()
+    P, Q = dd @ hxd, hgd @ dd
+    rel = lambda k: 1.5 * 2.0 ** -20 + 2 * math.sqrt(3 * k) * 2.0 ** -24 + 2.0 ** -23
+    bound = rel(d_in) * float(((dd.abs() @ hxd.abs()) * Q.abs()).sum()) + \
+        rel(d_out) * float((P.abs() * (hgd.abs() @ dd.abs())).sum())
+    assert abs(loss.item() - want) <= bound
+    assert math.isclose(loss.item(), want, rel_tol=1e-3)   # the method's bar
