@@ -275,17 +275,24 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
  *   A: M x K (a_mn = 0, pitch lda) or its transpose stored K x M (a_mn = 1),
  *   B: N x K (b_mn = 0, pitch ldb) or its transpose stored K x N (b_mn = 1),
  *   C: M x N, pitch ldc; beta = 0 ignores the old C.
- * Each fp32 operand is split into TF32 high and low parts and three MMAs
- * (hi*hi, hi*lo, lo*hi) accumulate in fp32. Pointers 16-byte aligned,
- * pitches multiples of 4 elements; M, N, K >= 0. C must not overlap A or B.
- * INVALID_ARG for negative sizes or null pointers, UNSUPPORTED for
- * misaligned operands, TIMEOUT in *info_dev (nonzero) if a pipeline wait
- * ran out.
+ * Each fp32 operand is split into a high and a low part and three MMAs
+ * (hi*hi, hi*lo, lo*hi) accumulate in fp32: TF32 parts, or, for large
+ * products when ws holds kronq_gemm_f32_workspace_bytes(M, N, K) bytes
+ * (device, 256-byte aligned, busy until the product completes on the stream),
+ * fp16 parts of the operand rows scaled by powers of two. ws may be NULL.
+ * Pointers 16-byte aligned, pitches multiples of 4 elements; M, N, K >= 0.
+ * C must not overlap A or B. INVALID_ARG for negative sizes or null
+ * pointers, UNSUPPORTED for misaligned operands, TIMEOUT in *info_dev
+ * (nonzero) if a pipeline wait ran out.
  */
 kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,
                             int64_t K, float alpha, const float *A, int64_t lda,
                             int a_mn, const float *B, int64_t ldb, int b_mn,
-                            float beta, float *C, int64_t ldc, int32_t *info_dev);
+                            float beta, float *C, int64_t ldc, void *ws,
+                            size_t ws_bytes, int32_t *info_dev);
+/* Workspace bytes that let kronq_gemm_f32 take the fp16 path (0 if M, N or
+ * K <= 0). */
+size_t kronq_gemm_f32_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Workspace bytes needed by one call (opts may be NULL except for BIIP and
  * QUANT). Returns 0 for unsupported arguments. */

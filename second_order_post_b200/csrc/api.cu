@@ -171,7 +171,8 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
 kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,
                             int64_t K, float alpha, const float *A, int64_t lda,
                             int a_mn, const float *B, int64_t ldb, int b_mn,
-                            float beta, float *C, int64_t ldc, int32_t *info_dev) {
+                            float beta, float *C, int64_t ldc, void *ws,
+                            size_t ws_bytes, int32_t *info_dev) {
   if (M < 0 || N < 0 || K < 0 || !info_dev) return KRONQ_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return KRONQ_OK;
   if (!C || (K > 0 && (!A || !B))) return KRONQ_ERR_INVALID_ARG;
@@ -200,7 +201,12 @@ kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,
   g.B = B; g.ldb = ldb; g.b_mn = b_mn != 0;
   g.C = C; g.ldc = ldc;
   g.alpha = alpha; g.beta = beta;
-  return gemm_tf32x3(st, g, info_dev);
+  if (ws && !aligned(ws, 256)) return KRONQ_ERR_INVALID_ARG;
+  return gemm_f32(st, g, ws, ws ? ws_bytes : 0, info_dev);
+}
+
+size_t kronq_gemm_f32_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return gemm_scratch_bytes(M, N, K);
 }
 
 kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,

@@ -235,6 +235,9 @@ struct Ctx {
   int64_t d;
   float *V[MAXD];            // B U22ᵀ of the node at each depth
   float *T[MAXD];            // V U22 of the node at each depth
+  void *scr_main;            // GEMM scratch of the critical path
+  void *scr_side[MAXD];      // and of each depth's side stream
+  size_t scr_main_bytes, scr_side_bytes[MAXD];
   const float *lambda;
   int32_t *info;
 };
@@ -303,7 +306,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.B = C22; g.ldb = d;
     g.C = V; g.ldc = m;
     g.kflags = KR_B_UPPER;
-    KQ_TRY(gemm_tf32x3(c.st, g, c.info));
+    KQ_TRY(gemm_f32(c.st, g, c.scr_main, c.scr_main_bytes, c.info));
   }
   // T = V U22 does not feed the recursion into A11: run it beside it
   if (cudaEventRecord(c.ev_v[depth], c.st) != cudaSuccess ||
@@ -316,7 +319,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.B = C22; g.ldb = d; g.b_mn = true;
     g.C = T; g.ldc = m;
     g.kflags = KR_B_LOWER;
-    KQ_TRY(gemm_tf32x3(c.side[depth], g, c.info));
+    KQ_TRY(gemm_f32(c.side[depth], g, c.scr_side[depth], c.scr_side_bytes[depth], c.info));
   }
   if (cudaEventRecord(c.ev_t[depth], c.side[depth]) != cudaSuccess)
     return KRONQ_ERR_CUDA;
@@ -328,7 +331,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.C = A11; g.ldc = d;
     g.alpha = -1.f; g.beta = 1.f;
     g.upper_tiles_only = true;
-    KQ_TRY(gemm_tf32x3(c.st, g, c.info));
+    KQ_TRY(gemm_f32(c.st, g, c.scr_main, c.scr_main_bytes, c.info));
   }
   KQ_TRY(rinv(c, off, h, depth + 1));  // A11 -> U11
   if (cudaStreamWaitEvent(c.st, c.ev_t[depth], 0) != cudaSuccess) return KRONQ_ERR_CUDA;
@@ -340,7 +343,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.C = B12; g.ldc = d;
     g.alpha = -1.f;
     g.kflags = KR_A_UPPER;
-    KQ_TRY(gemm_tf32x3(c.st, g, c.info));
+    KQ_TRY(gemm_f32(c.st, g, c.scr_main, c.scr_main_bytes, c.info));
   }
   // zeros below the diagonal of this node (the leaves zero their own blocks):
   // triangular operands of the parents' products read U as 128 x 256 tiles
@@ -351,10 +354,13 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
   return KRONQ_OK;
 }
 
-// Workspace layout: [V, T] slots per recursion depth, then lambda. The
-// largest node at depth i+1 is the larger child m_i of the largest node at i.
+// Workspace layout: [V, T, side-stream GEMM scratch] per recursion depth, the
+// critical path's GEMM scratch, then lambda. The largest node at depth i+1 is
+// the larger child m_i of the largest node at i, and the node sizes bound the
+// products' scratch (V: h x m x m, SYRK: h x h x m, U12: h x m x h, T: h x m x m).
 struct CholLayout {
-  size_t v[MAXD], t[MAXD];
+  size_t v[MAXD], t[MAXD], side[MAXD], side_bytes[MAXD];
+  size_t main, main_bytes;
   int depths;
   size_t total;
 };
@@ -362,17 +368,25 @@ CholLayout chol_layout(int64_t d) {
   auto al = [](size_t b) { return (b + 255) / 256 * 256; };
   CholLayout L{};
   size_t off = 0;
+  size_t main_bytes = 0;
   int k = 0;
   for (int64_t n = d; n > NB && k < MAXD; ++k) {
-    const int64_t h = first_half(n);
-    const size_t slot = al(static_cast<size_t>(h) * (n - h) * 4);
+    const int64_t h = first_half(n), m = n - h;
+    const size_t slot = al(static_cast<size_t>(h) * m * 4);
     L.v[k] = off;
     L.t[k] = off + slot;
-    off += 2 * slot;
-    n = n - h;
+    L.side[k] = off + 2 * slot;
+    L.side_bytes[k] = al(gemm_scratch_bytes(h, m, m));
+    off += 2 * slot + L.side_bytes[k];
+    main_bytes = kq_max(main_bytes, kq_max(gemm_scratch_bytes(h, m, m),
+                                           kq_max(gemm_scratch_bytes(h, h, m),
+                                                  gemm_scratch_bytes(h, m, h))));
+    n = m;
   }
   L.depths = k;
-  L.total = off + 256;
+  L.main = off;
+  L.main_bytes = al(main_bytes);
+  L.total = off + L.main_bytes + 256;
   return L;
 }
 
@@ -402,7 +416,11 @@ kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
     c.ev_t[k] = cs->ev_t[k];
     c.V[k] = at(k, lay.v[k]);
     c.T[k] = at(k, lay.t[k]);
+    c.scr_side[k] = at(k, lay.side[k]);
+    c.scr_side_bytes[k] = k < depths ? lay.side_bytes[k] : 0;
   }
+  c.scr_main = w + lay.main;
+  c.scr_main_bytes = lay.main_bytes;
   float *lambda = reinterpret_cast<float *>(w + need - 256);
   c.lambda = lambda;
   c.info = info;

@@ -34,6 +34,12 @@ struct GemmArgs {
 };
 
 kronq_status gemm_tf32x3(cudaStream_t st, const GemmArgs &g, int32_t *info);
+// Same product; large ones run on the fp16-split path when `scratch` holds at
+// least gemm_scratch_bytes(M, N, K) bytes (256-byte aligned), the rest on
+// gemm_tf32x3. The scratch is in use until the product completes on `st`.
+kronq_status gemm_f32(cudaStream_t st, const GemmArgs &g, void *scratch,
+                      size_t scratch_bytes, int32_t *info);
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
 // ---------------------------------------------------------------- covariance
 kronq_status cov_bf16(cudaStream_t st, const __nv_bfloat16 *A, int64_t n,

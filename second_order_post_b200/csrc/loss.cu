@@ -30,9 +30,11 @@ __global__ void dot_kernel(const float *p, const float *q, int64_t n, double *ou
 
 }  // namespace
 
+// Workspace: D, P, Q (d_out x d_in each), then scratch for the two products.
 size_t loss_ws_bytes(int64_t d_out, int64_t d_in) {
   const size_t one = (static_cast<size_t>(d_out) * d_in * 4 + 255) / 256 * 256;
-  return 3 * one + 256;
+  return 3 * one + kq_max(gemm_scratch_bytes(d_out, d_in, d_in),
+                          gemm_scratch_bytes(d_out, d_in, d_out)) + 256;
 }
 
 kronq_status layer_loss(cudaStream_t st, const float *W_ref, const float *W_hat,
@@ -44,6 +46,8 @@ kronq_status layer_loss(cudaStream_t st, const float *W_ref, const float *W_hat,
   float *D = reinterpret_cast<float *>(w);
   float *P = reinterpret_cast<float *>(w + one);
   float *Q = reinterpret_cast<float *>(w + 2 * one);
+  void *scr = w + 3 * one;
+  const size_t scr_bytes = ws_bytes - 3 * one;
   const int64_t n = d_out * d_in;
   const unsigned blocks = static_cast<unsigned>(kq_min<int64_t>(ceil_div(n, 256), 148 * 8));
   diff_kernel<<<blocks, 256, 0, st>>>(W_ref, W_hat, D, n);
@@ -53,13 +57,13 @@ kronq_status layer_loss(cudaStream_t st, const float *W_ref, const float *W_hat,
   g.A = D; g.lda = d_in;
   g.B = H_X; g.ldb = d_in;
   g.C = P; g.ldc = d_in;
-  KQ_TRY(gemm_tf32x3(st, g, nullptr));
+  KQ_TRY(gemm_f32(st, g, scr, scr_bytes, nullptr));
   GemmArgs h;  // Q = H_G D
   h.M = d_out; h.N = d_in; h.K = d_out;
   h.A = H_G; h.lda = d_out;
   h.B = D; h.ldb = d_in; h.b_mn = true;
   h.C = Q; h.ldc = d_in;
-  KQ_TRY(gemm_tf32x3(st, h, nullptr));
+  KQ_TRY(gemm_f32(st, h, scr, scr_bytes, nullptr));
   if (cudaMemsetAsync(loss, 0, sizeof(double), st) != cudaSuccess) return KRONQ_ERR_CUDA;
   dot_kernel<<<blocks, 256, 0, st>>>(P, Q, n, loss);
   KQ_CHECK_LAUNCH();

@@ -176,9 +176,12 @@ __global__ void __launch_bounds__(OTHREADS)
 
 }  // namespace
 
+// Workspace: the errors E (d_out x S), then scratch for the super-block
+// products (d_out x (d_in - S) x S at most).
 size_t quant_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &) {
   const int64_t S = kq_min<int64_t>(d_in, SUPER);
-  return static_cast<size_t>(d_out) * S * 4 + 256;
+  const size_t e = (static_cast<size_t>(d_out) * S * 4 + 255) / 256 * 256;
+  return e + gemm_scratch_bytes(d_out, d_in - S, S) + 256;
 }
 
 kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
@@ -188,6 +191,9 @@ kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
   if (ws_bytes < quant_ws_bytes(d_out, d_in, o)) return KRONQ_ERR_INVALID_ARG;
   const int64_t S = kq_min<int64_t>(d_in, SUPER);
   float *E = static_cast<float *>(ws);
+  const size_t e_bytes = (static_cast<size_t>(d_out) * S * 4 + 255) / 256 * 256;
+  void *scr = static_cast<uint8_t *>(ws) + e_bytes;
+  const size_t scr_bytes = ws_bytes - e_bytes;
   const int64_t ngroups = d_in / o.group;
   const int64_t ldq = o.bits * d_in / 32;
   static bool attr_done = false;
@@ -223,7 +229,7 @@ kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
       g.B = U + sb0 * d_in + sb1; g.ldb = d_in; g.b_mn = true;
       g.C = W + sb1; g.ldc = d_in;
       g.alpha = -1.f; g.beta = 1.f;
-      KQ_TRY(gemm_tf32x3(st, g, info));
+      KQ_TRY(gemm_f32(st, g, scr, scr_bytes, info));
     }
   }
   return KRONQ_OK;

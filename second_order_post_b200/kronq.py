@@ -79,7 +79,8 @@ _SIGS = {
                                 _sz, _p],
     "kronq_layer_loss": [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _sz],
     "kronq_gemm_f32": [_p, _i64, _i64, _i64, _f, _p, _i64, ctypes.c_int, _p,
-                       _i64, ctypes.c_int, _f, _p, _i64, _p],
+                       _i64, ctypes.c_int, _f, _p, _i64, _p, _sz, _p],
+    "kronq_gemm_f32_workspace_bytes": [_i64, _i64, _i64],
     "kronq_workspace_bytes": [ctypes.c_int, _i64, _i64, _OPTS],
     "kronq_allocate_bits": [_p, _p, ctypes.c_int, _d, _p],
     "kronq_status_string": [ctypes.c_int],
@@ -90,6 +91,7 @@ for _name, _args in _SIGS.items():
     _fn.argtypes = _args
     _fn.restype = ctypes.c_int
 _lib.kronq_workspace_bytes.restype = ctypes.c_size_t
+_lib.kronq_gemm_f32_workspace_bytes.restype = ctypes.c_size_t
 _lib.kronq_status_string.restype = ctypes.c_char_p
 _lib.kronq_kernel_launches.restype = ctypes.c_uint64
 
@@ -179,14 +181,21 @@ def kronq_layer_loss(W_ref, W_hat, H_X, H_G, loss, ws, stream=None):
 
 
 def kronq_gemm_f32(A, B, C, info, alpha=1.0, beta=0.0, a_mn=False, b_mn=False,
-                   stream=None):
+                   ws=None, stream=None):
     """C = alpha * A Bᵀ + beta * C; A is M x K (or K x M with a_mn), B is
-    N x K (or K x N with b_mn); all 2-D fp32 CUDA tensors, rows contiguous."""
+    N x K (or K x N with b_mn); all 2-D fp32 CUDA tensors, rows contiguous.
+    ws (a uint8 CUDA tensor) lets large products take the fp16-split path."""
     M, N = C.shape
     K = A.shape[0] if a_mn else A.shape[1]
     _check("kronq_gemm_f32", _lib.kronq_gemm_f32(
         _stream(stream), M, N, K, alpha, _ptr(A), A.stride(0), int(a_mn),
-        _ptr(B), B.stride(0), int(b_mn), beta, _ptr(C), C.stride(0), _ptr(info)))
+        _ptr(B), B.stride(0), int(b_mn), beta, _ptr(C), C.stride(0),
+        None if ws is None else _ptr(ws), 0 if ws is None else ws.numel(),
+        _ptr(info)))
+
+
+def kronq_gemm_f32_workspace_bytes(M, N, K):
+    return _lib.kronq_gemm_f32_workspace_bytes(M, N, K)
 
 
 def kronq_allocate_bits(scores, numel, avg_budget):

@@ -66,12 +66,18 @@ def test_invalid_args_rejected_before_device(K):
     # gemm: negative sizes, short pitches, misalignment, C overlapping A
     g = lib.kronq_gemm_f32
     q = ctypes.c_void_p(1 << 20)
-    assert g(None, -1, 8, 8, 1.0, p, 8, 0, p, 8, 0, 0.0, q, 8, p) == K.KRONQ_ERR_INVALID_ARG
-    assert g(None, 8, 8, 8, 1.0, p, 4, 0, p, 8, 0, 0.0, q, 8, p) == K.KRONQ_ERR_INVALID_ARG
+    assert g(None, -1, 8, 8, 1.0, p, 8, 0, p, 8, 0, 0.0, q, 8, None, 0, p) == \
+        K.KRONQ_ERR_INVALID_ARG
+    assert g(None, 8, 8, 8, 1.0, p, 4, 0, p, 8, 0, 0.0, q, 8, None, 0, p) == \
+        K.KRONQ_ERR_INVALID_ARG
     assert g(None, 8, 8, 8, 1.0, ctypes.c_void_p(260), 8, 0, p, 8, 0, 0.0, q, 8,
-             p) == K.KRONQ_ERR_UNSUPPORTED
-    assert g(None, 8, 8, 8, 1.0, p, 8, 0, q, 8, 0, 0.0, p, 8, p) == K.KRONQ_ERR_INVALID_ARG
-    assert g(None, 0, 8, 8, 1.0, nullp, 8, 0, nullp, 8, 0, 0.0, nullp, 8, p) == K.KRONQ_OK
+             None, 0, p) == K.KRONQ_ERR_UNSUPPORTED
+    assert g(None, 8, 8, 8, 1.0, p, 8, 0, q, 8, 0, 0.0, p, 8, None, 0, p) == \
+        K.KRONQ_ERR_INVALID_ARG
+    assert g(None, 0, 8, 8, 1.0, nullp, 8, 0, nullp, 8, 0, 0.0, nullp, 8, None, 0,
+             p) == K.KRONQ_OK
+    assert K.kronq_gemm_f32_workspace_bytes(0, 8, 8) == 0
+    assert K.kronq_gemm_f32_workspace_bytes(256, 512, 1024) >= 4 * (256 + 512) * 1024
 
 
 def test_workspace_sizes(K):

@@ -273,10 +273,12 @@ GEMM_CASES = [(300, 200, 100, 0, 0), (256, 384, 1000, 1, 0), (129, 132, 64, 0, 1
               (1920, 3968, 2080, 0, 1), (4096, 2816, 512, 1, 0)]
 
 
+@pytest.mark.parametrize("split", ["tf32", "fp16"])
 @pytest.mark.parametrize("case", GEMM_CASES)
-def test_gemm_f32(cuda_device, case):
+def test_gemm_f32(cuda_device, case, split):
     """Elementwise against fp64. Each product keeps all but
-    1.5 * 2^-20 |a b| (truncated hi, rounded lo, no lo*lo term) and the
+    1.5 * 2^-20 |a b| (TF32: truncated hi, rounded lo, no lo*lo term; the
+    fp16 split of row-scaled operands keeps about 3 * 2^-22) and the
     3K/8 fp32 accumulation steps add rounding that grows like their square
     root: |err| <= (1.5 * 2^-20 + 2 sqrt(3K) 2^-24) |alpha| (|A| |B|^T)
     plus one rounding of the result. A missing or misplaced hi/lo term
@@ -292,7 +294,11 @@ def test_gemm_f32(cuda_device, case):
     B = b.T.contiguous() if b_mn else b
     C = c0.clone()
     info = torch.ones(1, dtype=torch.int32, device="cuda")
-    Kq.kronq_gemm_f32(A, B, C, info, alpha=-0.5, beta=2.0, a_mn=a_mn, b_mn=b_mn)
+    ws = None
+    if split == "fp16":   # large products take the fp16 path given a workspace
+        ws = torch.empty(Kq.kronq_gemm_f32_workspace_bytes(M, N, Kd), dtype=torch.uint8,
+                         device="cuda")
+    Kq.kronq_gemm_f32(A, B, C, info, alpha=-0.5, beta=2.0, a_mn=a_mn, b_mn=b_mn, ws=ws)
     torch.cuda.synchronize()
     assert info.item() == 0
     want = 2.0 * c0.double() - 0.5 * (a.double() @ b.double().T)
