@@ -154,7 +154,12 @@ def sensitivity(h_x: np.ndarray, h_g: np.ndarray):
 # --------------------------------------------------------------------------
 def diag_scale(h: np.ndarray, exponent: float) -> np.ndarray:
     """s_i = max(h_ii, 1e-8·mean(diag h))^exponent (reading of wmrh §八)."""
-    dg = np.diag(np.asarray(h, dtype=np.float64)).copy()
+    return diag_scale_of(np.diag(np.asarray(h, dtype=np.float64)), exponent)
+
+
+def diag_scale_of(dg: np.ndarray, exponent: float) -> np.ndarray:
+    """diag_scale from the diagonal alone (for sizes where H is not kept)."""
+    dg = np.asarray(dg, dtype=np.float64).copy()
     floor = 1e-8 * dg.mean()
     return np.maximum(dg, floor) ** exponent
 

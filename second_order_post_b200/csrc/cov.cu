@@ -7,10 +7,18 @@
 // streams the n rows of A through a 3-stage TMA ring, 64 rows per stage. Both
 // MMA operands are the same row slab of A read feature-contiguous
 // ("MN-major"), so A is consumed in place without a transpose. Only tiles on
-// or above the diagonal are computed; the epilogue writes each value to (i,j)
-// and to its mirror (j,i), so both triangles are bitwise equal. Tiles are
-// visited in 12x12 super-tiles so that the CTAs resident at one time touch a
-// small set of feature columns and share each A slab through L2.
+// or above the diagonal are computed; each value ends in (i,j) and in its
+// mirror (j,i), so both triangles are bitwise equal. Tiles are visited in
+// 12x12 super-tiles so that the CTAs resident at one time touch a small set
+// of feature columns and share each A slab through L2.
+//
+// The tensor core's fp32 accumulation loses part of an ulp per step in one
+// direction (measured: a sum of 131072 squares comes out 6.6e-4 low when
+// accumulated in TMEM alone). The accumulator therefore restarts every
+// CHUNK rows of A: eight epilogue warps fold each chunk's sum into H with
+// round-to-nearest fp32 adds (through the mirror (j,i), whose addresses are
+// consecutive across a warp's lanes) while the MMA waits, and the last fold
+// writes both triangles. A chunk of 8192 rows keeps the drift near 4e-5.
 //
 // fp32 path: plain FFMA tiles (used for fp32 calibration data).
 #include "kernels.cuh"
@@ -23,13 +31,16 @@ constexpr int CBK = 64;               // rows of A per stage
 constexpr int CSTAGES = 3;
 constexpr int CBOX = 64 * CBK * 2;    // one TMA box: 64 rows x 64 features bf16
 constexpr int CSTAGE_BYTES = 8 * CBOX;  // 4 boxes for the row panel, 4 for the column panel
-constexpr int CTHREADS = 256;
+constexpr int CTHREADS = 320;         // TMA warp, MMA warp, 8 epilogue warps
 constexpr int SUPER = 12;
+constexpr int CHUNK = 8192;           // rows of A per TMEM accumulation
+constexpr int CHUNK_K = CHUNK / CBK;  // stages per chunk
 
 struct CovCtl {
   uint64_t full[CSTAGES];
   uint64_t empty[CSTAGES];
-  uint64_t done;
+  uint64_t chunk_done;  // MMAs of a chunk finished (commit)
+  uint64_t folded;      // the epilogue warps have read the accumulator (256)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -92,7 +103,8 @@ __global__ void __launch_bounds__(CTHREADS, 1)
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    mbar_init(&ctl->done, 1);
+    mbar_init(&ctl->chunk_done, 1);
+    mbar_init(&ctl->folded, 256);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -131,6 +143,9 @@ __global__ void __launch_bounds__(CTHREADS, 1)
     const uint32_t idesc = idesc_make(1, 1, 1, 128, 256);
     for (int it = 0; it < nk; ++it) {
       const int s = it % CSTAGES;
+      const int ci = it / CHUNK_K, first = it % CHUNK_K == 0;
+      // a new chunk overwrites the accumulator once the last one is folded
+      if (first && ci > 0 && !mbar_wait(&ctl->folded, (ci - 1) & 1, abort)) break;
       if (!mbar_wait(&ctl->full[s], (it / CSTAGES) & 1, abort)) break;
       tc_fence_after();
       const uint32_t a0 = smem_u32(smem + s * CSTAGE_BYTES);
@@ -141,47 +156,48 @@ __global__ void __launch_bounds__(CTHREADS, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint64_t da = sdesc_sw128(a0 + h * 2 * CBOX + kk * 2048, CBOX, 1024);
-          umma_bf16(tbase + 256 * h, da, db, idesc, (it | kk) != 0);
+          umma_bf16(tbase + 256 * h, da, db, idesc, (!first || kk != 0) ? 1u : 0u);
         }
       }
       umma_commit(&ctl->empty[s]);
+      if (it % CHUNK_K == CHUNK_K - 1 || it == nk - 1) umma_commit(&ctl->chunk_done);
     }
-    if (nk > 0)
-      umma_commit(&ctl->done);
-    else
-      mbar_arrive(&ctl->done);
+  } else if (warp >= 2) {
+    // ---- epilogue warps: warp w folds accumulator (w-2)/4, TMEM lanes
+    // 32*(w%4) .. +31 (tile rows), all 256 columns of its half
+    const int h = (warp - 2) >> 2, q = warp & 3;
+    const int64_t i = i0 + 128 * h + 32 * q + lane;
+    const bool diag = (bi == bj);
+    const int nchunks = nk > 0 ? (nk + CHUNK_K - 1) / CHUNK_K : 0;
+    for (int ci = 0; ci < nchunks; ++ci) {
+      const bool ok = mbar_wait(&ctl->chunk_done, ci & 1, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const bool last = ci == nchunks - 1;
+      for (int c = 0; c < CT / 32; ++c) {
+        float v[32];
+        tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 256 * h + 32 * c, v);
+        const int64_t jc = j0 + 32 * c;
+        if (jc >= d) continue;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const int64_t j = jc + t;
+          if (!((i < d) && (j < d) && (!diag || j >= i))) continue;
+          float o = alpha * v[t];
+          const float prev = H[j * d + i];  // running sum (or old H) at the mirror
+          if (ci > 0) o += prev;
+          else if (beta != 0.f) o += beta * prev;
+          H[j * d + i] = o;
+          if (last && j != i) H[i * d + j] = o;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->folded);
+    }
+    if (nchunks == 0) {  // n == 0 never reaches here (host scales H instead)
+    }
   }
   __syncwarp();
-
-  // ---- epilogue (all 8 warps): warp w reads accumulator w/4, lanes 32*(w%4)..
-  const bool ok = mbar_wait(&ctl->done, 0, abort);
-  const bool have = __all_sync(0xffffffffu, ok) && nk > 0;
-  tc_fence_after();
-  const int h = warp >> 2, q = warp & 3;
-  const int64_t i = i0 + 128 * h + 32 * q + lane;
-  const bool diag = (bi == bj);
-  for (int c = 0; c < CT / 32; ++c) {
-    float v[32];
-    if (have) {
-      tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 256 * h + 32 * c, v);
-    } else {
-#pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] = 0.f;
-    }
-    const int64_t jc = j0 + 32 * c;
-    if (jc >= d) continue;
-#pragma unroll 4
-    for (int t = 0; t < 32; ++t) {
-      const int64_t j = jc + t;
-      const bool in = (i < d) && (j < d) && (!diag || j >= i);
-      float o = alpha * v[t];
-      if (in && beta != 0.f) o += beta * H[i * d + j];
-      if (in) {
-        H[i * d + j] = o;
-        if (j != i) H[j * d + i] = o;
-      }
-    }
-  }
 
   tc_fence_before();
   __syncthreads();

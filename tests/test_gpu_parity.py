@@ -20,6 +20,7 @@ import pytest
 import torch
 
 import oracle as O
+from parity_helpers import replay_check
 from second_order_post_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -46,8 +47,11 @@ def dev(x, dtype=None):
 
 
 # ------------------------------------------------------------------ covariance
+# 131072 rows (the 70B down_proj calibration size) and a ragged 139264 run
+# over many accumulator restarts; the diagonal (sums of squares, all terms of
+# one sign) is where accumulation drift would show first
 @pytest.mark.parametrize("n,d", [(64, 128), (1000, 256), (777, 384), (4096, 1024),
-                                 (8192, 4096)])
+                                 (8192, 4096), (131072, 512), (139200, 256)])
 def test_cov_bf16(cuda_device, n, d):
     X = synth.make_activations(n, d, -1, 1, torch.bfloat16, seed=n + d)
     H = torch.empty(d, d, device="cuda")
@@ -56,6 +60,7 @@ def test_cov_bf16(cuda_device, n, d):
     want = O.cov(X.float().numpy())
     got = f64(H)
     assert rel_fro(got, want) < 1e-4
+    assert np.abs(np.diag(got) / np.diag(want) - 1).max() < 1e-4
     assert torch.equal(H, H.T)                      # both triangles bitwise equal
 
 
@@ -176,25 +181,6 @@ def test_chol_inv_reports_not_pd(cuda_device):
 
 
 # ------------------------------------------------------------------ OBS
-def replay_check(w, u, codes, zeros, bits, group, tau=1e-3):
-    """Every decision of a candidate must be the oracle's rounding of the
-    value it sees given the candidate's own earlier decisions, except within
-    tau of a rounding tie. Returns (fraction identical to that decision,
-    number of non-tie mismatches, number of tie mismatches)."""
-    rep = O.obs_quantize(w, u, bits, group, forced_codes=codes, forced_zeros=zeros)
-    maxq = 2 ** bits - 1
-    v = rep["v"]
-    frac = v - np.floor(v)
-    near_tie = np.abs(frac - 0.5) < tau
-    near_clamp = (np.abs(v - (maxq + 0.5)) < tau) | (np.abs(v + 0.5) < tau)
-    mism = codes != rep["own"]
-    bad = mism & ~(near_tie | near_clamp)
-    # zero points: rint(-xmin/scale) may differ only at a tie
-    zr = rep["zraw"]
-    zbad = (zeros != np.rint(zr)) & ~(np.abs(zr - np.floor(zr) - 0.5) < tau)
-    return 1.0 - mism.mean(), int(bad.sum()) + int(zbad.sum()), int((mism & ~bad).sum())
-
-
 def _quant_inputs(d_out, d_in, seed):
     data = synth.small_case(d_out, d_in, 2 * d_in, seed=seed)
     w = data["W"].double().numpy()
