@@ -33,6 +33,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int NTHREADS = 192;
 constexpr int GROUP_M = 16;                    // tile raster: 16 rows per band
+constexpr int KCHUNK = 4096;                   // k per main-accumulator chunk
 
 template <int STAGES>
 struct Ctl {
@@ -40,6 +41,8 @@ struct Ctl {
   uint64_t conv[STAGES];   // hi/lo split written (128 arrivals)
   uint64_t empty[STAGES];  // MMAs that read the stage finished (commit)
   uint64_t done;           // all MMAs finished (commit)
+  uint64_t chunk_done;     // hi*hi MMAs of a k-chunk finished (commit)
+  uint64_t folded;         // epilogue warps read the main accumulator (128)
   uint64_t drain;          // teardown drain after an abort
   uint32_t tmem_base;
   int abort;
@@ -63,6 +66,7 @@ struct Cfg {
   static constexpr uint32_t K_SBO = 8 * BK * ES;   // 8-row group
   static constexpr uint32_t MN_CHUNK = BK * 128;   // one 32-wide MN chunk
   static constexpr int KSTEP = F16 ? 16 : 8;       // K of one MMA (32 bytes)
+  static constexpr int CH = KCHUNK / BK;           // stages per k-chunk
   static_assert(BK * ES == 128 || BK * ES == 64, "k-slab rows of 64 or 128 bytes");
   static_assert(BN == 128 || BN == 256, "tile width");
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -142,6 +146,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&ctl->empty[s], 1);
     }
     mbar_init(&ctl->done, 1);
+    mbar_init(&ctl->chunk_done, 1);
+    mbar_init(&ctl->folded, 128);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -153,7 +159,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, BN);
+    tmem_alloc(&ctl->tmem_base, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -209,9 +215,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t lbo_b = b_mn ? C::MN_CHUNK : 16;
       const uint32_t sbo_a = a_mn ? 512 : C::K_SBO, sbo_b = b_mn ? 512 : C::K_SBO;
       const uint32_t lay_a = a_mn ? 1 : C::K_LAYOUT, lay_b = b_mn ? 1 : C::K_LAYOUT;
-      int it = 0;
-      for (; it < nk; ++it) {
+      // hi*hi into the main accumulator (columns [0, BN)), restarted every
+      // k-chunk after the epilogue warps folded it into C; the two cross
+      // terms into a second accumulator (columns [BN, 2 BN)) that runs over
+      // all of K (its one-way rounding drift is relative to a value ~2^-11
+      // the size of the main one)
+      for (int it = 0; it < nk; ++it) {
         const int s = it % STAGES;
+        const int ci = it / C::CH, first = it % C::CH == 0;
+        if (first && ci > 0 && !mbar_wait(&ctl->folded, (ci - 1) & 1, abort)) break;
         if (!mbar_wait(C::F16 ? &ctl->full[s] : &ctl->conv[s], (it / STAGES) & 1, abort))
           break;
         tc_fence_after();
@@ -227,17 +239,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint64_t dal = sdesc(a_lo + ao, lbo_a, sbo_a, lay_a);
           const uint64_t dbh = sdesc(b_hi + bo, lbo_b, sbo_b, lay_b);
           const uint64_t dbl = sdesc(b_lo + bo, lbo_b, sbo_b, lay_b);
+          const uint32_t cross = (it | kk) != 0, main = !(first && kk == 0);
           if (C::F16) {
-            umma_bf16(tbase, dal, dbh, idesc, (it | kk) != 0);
-            umma_bf16(tbase, dah, dbl, idesc, 1);
-            umma_bf16(tbase, dah, dbh, idesc, 1);
+            umma_bf16(tbase + BN, dal, dbh, idesc, cross);
+            umma_bf16(tbase + BN, dah, dbl, idesc, 1);
+            umma_bf16(tbase, dah, dbh, idesc, main);
           } else {
-            umma_tf32(tbase, dal, dbh, idesc, (it | kk) != 0);
-            umma_tf32(tbase, dah, dbl, idesc, 1);
-            umma_tf32(tbase, dah, dbh, idesc, 1);
+            umma_tf32(tbase + BN, dal, dbh, idesc, cross);
+            umma_tf32(tbase + BN, dah, dbl, idesc, 1);
+            umma_tf32(tbase, dah, dbh, idesc, main);
           }
         }
         umma_commit(&ctl->empty[s]);
+        if (it % C::CH == C::CH - 1 && it != nk - 1) umma_commit(&ctl->chunk_done);
       }
       if (nk > 0)
         umma_commit(&ctl->done);
@@ -245,77 +259,106 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&ctl->done);
     }
   } else {
-    // ---- hi/lo split of every landed slab
     const int ct = threadIdx.x - 64;
-    for (int it = 0; it < (C::F16 ? 0 : nk); ++it) {
-      const int s = it % STAGES;
-      if (!mbar_wait(&ctl->full[s], (it / STAGES) & 1, abort)) break;
-      float4 *sa = reinterpret_cast<float4 *>(smem + s * C::STAGE);
-      float4 *sb = sa + 2 * (TA / 16);
-      // all loads first: the slabs and their low parts share one array
-      float4 ra[TA / 16 / 128], rb[TB / 16 / 128];
-#pragma unroll
-      for (int j = 0; j < TA / 16 / 128; ++j) ra[j] = sa[ct + 128 * j];
-#pragma unroll
-      for (int j = 0; j < TB / 16 / 128; ++j) rb[j] = sb[ct + 128 * j];
-#pragma unroll
-      for (int j = 0; j < TA / 16 / 128; ++j) sa[TA / 16 + ct + 128 * j] = tf32_lo(ra[j]);
-#pragma unroll
-      for (int j = 0; j < TB / 16 / 128; ++j) sb[TB / 16 + ct + 128 * j] = tf32_lo(rb[j]);
-      fence_proxy_async_smem();
-      mbar_arrive(&ctl->conv[s]);
-    }
-    // ---- epilogue: TMEM lanes 32q..32q+31 hold tile rows 32q..32q+31
-    const bool ok = mbar_wait(&ctl->done, 0, abort);
-    const bool have = __all_sync(0xffffffffu, ok) && nk > 0;
-    tc_fence_after();
     const int q = warp & 3;
     const int64_t row = m0 + 32 * q + lane;
-    for (int c = 0; c < BN / 32; ++c) {
-      const int64_t col0 = n0 + 32 * c;
-      if (col0 >= N) break;
-      float v[32];
-      if (have) {
-        tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 32 * c, v);
-      } else {
+    int folds = 0;
+    // C (+)= the main accumulator (and, at the end, the cross terms): the first
+    // write applies beta to the old C, later ones add to what is there
+    auto fold = [&](bool final) -> bool {
+      const bool ok = mbar_wait(final ? &ctl->done : &ctl->chunk_done,
+                                final ? 0u : static_cast<uint32_t>(folds & 1), abort);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      tc_fence_after();
+      for (int c = 0; c < BN / 32; ++c) {
+        const int64_t col0 = n0 + 32 * c;
+        if (col0 >= N) break;
+        float v[32];
+        if (nk > 0) {
+          const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + 32 * c;
+          tmem_ld32(ta, v);
+          if (final) {
+            float u[32];
+            tmem_ld32(ta + BN, u);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] = 0.f;
-      }
-      if (row >= M) continue;
-      if (C::F16) {  // divide the operand row scales out
-        const float ra = p.alpha * p.inv_sa[row];
-#pragma unroll
-        for (int t = 0; t < 32; ++t)
-          v[t] *= ra * (col0 + t < N ? p.inv_sb[col0 + t] : 0.f);
-      } else {
-#pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] *= p.alpha;
-      }
-      float *crow = p.C + row * p.ldc + col0;
-      if (p.vec_ok && col0 + 32 <= N) {
-#pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          float4 o = make_float4(v[t], v[t + 1], v[t + 2], v[t + 3]);
-          if (p.beta != 0.f) {
-            const float4 old = *reinterpret_cast<const float4 *>(crow + t);
-            o.x += p.beta * old.x;
-            o.y += p.beta * old.y;
-            o.z += p.beta * old.z;
-            o.w += p.beta * old.w;
+            for (int t = 0; t < 32; ++t) v[t] += u[t];
           }
-          *reinterpret_cast<float4 *>(crow + t) = o;
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          if (col0 + t < N) {
-            float o = v[t];
-            if (p.beta != 0.f) o += p.beta * crow[t];
-            crow[t] = o;
+          for (int t = 0; t < 32; ++t) v[t] = 0.f;
+        }
+        if (row >= M) continue;
+        if (C::F16) {  // divide the operand row scales out
+          const float ra = p.alpha * p.inv_sa[row];
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            v[t] *= ra * (col0 + t < N ? p.inv_sb[col0 + t] : 0.f);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] *= p.alpha;
+        }
+        float *crow = p.C + row * p.ldc + col0;
+        const bool fresh = folds == 0, keep = !fresh || p.beta != 0.f;
+        const float bw = fresh ? p.beta : 1.f;
+        if (p.vec_ok && col0 + 32 <= N) {
+#pragma unroll
+          for (int t = 0; t < 32; t += 4) {
+            float4 o = make_float4(v[t], v[t + 1], v[t + 2], v[t + 3]);
+            if (keep) {
+              const float4 old = *reinterpret_cast<const float4 *>(crow + t);
+              o.x += bw * old.x;
+              o.y += bw * old.y;
+              o.z += bw * old.z;
+              o.w += bw * old.w;
+            }
+            *reinterpret_cast<float4 *>(crow + t) = o;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            if (col0 + t < N) {
+              float o = v[t];
+              if (keep) o += bw * crow[t];
+              crow[t] = o;
+            }
           }
         }
       }
+      tc_fence_before();
+      if (!final) mbar_arrive(&ctl->folded);
+      ++folds;
+      return true;
+    };
+    bool alive = true;
+    if (!C::F16) {
+      // ---- hi/lo split of every landed slab, folding each finished chunk
+      for (int it = 0; it < nk; ++it) {
+        if (it > 0 && it % C::CH == 0 && !fold(false)) {
+          alive = false;
+          break;
+        }
+        const int s = it % STAGES;
+        if (!mbar_wait(&ctl->full[s], (it / STAGES) & 1, abort)) break;
+        float4 *sa = reinterpret_cast<float4 *>(smem + s * C::STAGE);
+        float4 *sb = sa + 2 * (TA / 16);
+        // all loads first: the slabs and their low parts share one array
+        float4 ra[TA / 16 / 128], rb[TB / 16 / 128];
+#pragma unroll
+        for (int j = 0; j < TA / 16 / 128; ++j) ra[j] = sa[ct + 128 * j];
+#pragma unroll
+        for (int j = 0; j < TB / 16 / 128; ++j) rb[j] = sb[ct + 128 * j];
+#pragma unroll
+        for (int j = 0; j < TA / 16 / 128; ++j) sa[TA / 16 + ct + 128 * j] = tf32_lo(ra[j]);
+#pragma unroll
+        for (int j = 0; j < TB / 16 / 128; ++j) sb[TB / 16 + ct + 128 * j] = tf32_lo(rb[j]);
+        fence_proxy_async_smem();
+        mbar_arrive(&ctl->conv[s]);
+      }
+    } else {
+      const int nchunks = nk > 0 ? (nk + C::CH - 1) / C::CH : 0;
+      for (int c = 0; c + 1 < nchunks && alive; ++c) alive = fold(false);
     }
+    if (alive) fold(true);
   }
 
   // ---- teardown: after an abort make sure no copy or MMA is still in flight
@@ -342,7 +385,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, BN);
+    tmem_dealloc(tbase, 2 * BN);
   }
 }
 

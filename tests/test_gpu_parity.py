@@ -260,6 +260,33 @@ GEMM_CASES = [(300, 200, 100, 0, 0), (256, 384, 1000, 1, 0), (129, 132, 64, 0, 1
 
 
 @pytest.mark.parametrize("split", ["tf32", "fp16"])
+def test_gemm_f32_positive_long_k(cuda_device, split):
+    """Sums whose terms all have one sign (a Gram diagonal, as in the
+    Cholesky's Schur updates) over a long K: a one-way drift of the
+    tensor-core accumulation (up to one unit in the last place per MMA step)
+    adds up here instead of cancelling. The main accumulator restarts every
+    4096 k and the cross terms accumulate apart, so the drift stays below one
+    chunk's steps: (4096 / k-per-MMA) * 2^-23."""
+    Kq = K()
+    M, N, Kd = 4096, 4096, 16384
+    g = torch.Generator(device="cuda").manual_seed(7)
+    a = torch.randn(M, Kd, device="cuda", generator=g).abs()
+    C = torch.zeros(M, N, device="cuda")
+    info = torch.ones(1, dtype=torch.int32, device="cuda")
+    ws = None
+    if split == "fp16":
+        ws = torch.empty(Kq.kronq_gemm_f32_workspace_bytes(M, N, Kd), dtype=torch.uint8,
+                         device="cuda")
+    Kq.kronq_gemm_f32(a, a, C, info, ws=ws)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    want = a.double() @ a.double().T
+    rel = float(((C.double() - want) / want).abs().max())
+    kstep = 16 if split == "fp16" else 8
+    assert rel < (4096 // kstep) * 2.0 ** -23, rel
+
+
+@pytest.mark.parametrize("split", ["tf32", "fp16"])
 @pytest.mark.parametrize("case", GEMM_CASES)
 def test_gemm_f32(cuda_device, case, split):
     """Elementwise against fp64. Each product keeps all but
