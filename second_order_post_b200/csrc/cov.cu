@@ -18,7 +18,8 @@
 // CHUNK rows of A: eight epilogue warps fold each chunk's sum into H with
 // round-to-nearest fp32 adds (through the mirror (j,i), whose addresses are
 // consecutive across a warp's lanes) while the MMA waits, and the last fold
-// writes both triangles. A chunk of 8192 rows keeps the drift near 4e-5.
+// writes both triangles. A chunk of 16384 rows keeps the drift near 5e-5
+// (the measured loss is about 0.9 ulp per MMA step of 16 rows).
 //
 // fp32 path: plain FFMA tiles (used for fp32 calibration data).
 #include "kernels.cuh"
@@ -33,7 +34,7 @@ constexpr int CBOX = 64 * CBK * 2;    // one TMA box: 64 rows x 64 features bf16
 constexpr int CSTAGE_BYTES = 8 * CBOX;  // 4 boxes for the row panel, 4 for the column panel
 constexpr int CTHREADS = 320;         // TMA warp, MMA warp, 8 epilogue warps
 constexpr int SUPER = 12;
-constexpr int CHUNK = 8192;           // rows of A per TMEM accumulation
+constexpr int CHUNK = 16384;          // rows of A per TMEM accumulation
 constexpr int CHUNK_K = CHUNK / CBK;  // stages per chunk
 
 struct CovCtl {
@@ -161,6 +162,15 @@ __global__ void __launch_bounds__(CTHREADS, 1)
       }
       umma_commit(&ctl->empty[s]);
       if (it % CHUNK_K == CHUNK_K - 1 || it == nk - 1) umma_commit(&ctl->chunk_done);
+      // the fold of this chunk reads the running sums (rows j of the mirror
+      // block): bring them back into L2, which the streamed rows of A evicted
+      const bool fold_reads = ci > 0 || beta != 0.f;
+      if (fold_reads && (it % CHUNK_K == CHUNK_K - 8 || (it == nk - 8 && nk >= 8))) {
+        const int64_t cols = kq_min<int64_t>(CT, d - i0);
+        const uint32_t bytes = static_cast<uint32_t>(cols * 4) & ~15u;
+        for (int64_t j = j0; j < kq_min<int64_t>(j0 + CT, d) && bytes > 0; ++j)
+          prefetch_l2_bulk(H + j * d + i0, bytes);
+      }
     }
   } else if (warp >= 2) {
     // ---- epilogue warps: warp w folds accumulator (w-2)/4, TMEM lanes
@@ -179,14 +189,26 @@ __global__ void __launch_bounds__(CTHREADS, 1)
         tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 256 * h + 32 * c, v);
         const int64_t jc = j0 + 32 * c;
         if (jc >= d) continue;
+        // running sum (or the old H) at the mirror: all 32 loads before any
+        // store (their addresses are d apart, which the compiler cannot
+        // separate from the stores)
+        const bool need = ci > 0 || beta != 0.f;  // uniform across the CTA
+        const float bw = ci > 0 ? 1.f : beta;
+        float prev[32];
+        if (need) {  // unconditional loads at clamped (in-bounds) addresses
+          const int64_t ic = kq_min<int64_t>(i, d - 1);
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            prev[t] = __ldcg(H + kq_min<int64_t>(jc + t, d - 1) * d + ic);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) prev[t] = 0.f;
+        }
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
           const int64_t j = jc + t;
           if (!((i < d) && (j < d) && (!diag || j >= i))) continue;
-          float o = alpha * v[t];
-          const float prev = H[j * d + i];  // running sum (or old H) at the mirror
-          if (ci > 0) o += prev;
-          else if (beta != 0.f) o += beta * prev;
+          const float o = fmaf(bw, prev[t], alpha * v[t]);
           H[j * d + i] = o;
           if (last && j != i) H[i * d + j] = o;
         }

@@ -33,7 +33,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int NTHREADS = 192;
 constexpr int GROUP_M = 16;                    // tile raster: 16 rows per band
-constexpr int KCHUNK = 4096;                   // k per main-accumulator chunk
+constexpr int KCHUNK = 8192;                   // k per main-accumulator chunk
 
 template <int STAGES>
 struct Ctl {
@@ -301,17 +301,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const bool fresh = folds == 0, keep = !fresh || p.beta != 0.f;
         const float bw = fresh ? p.beta : 1.f;
         if (p.vec_ok && col0 + 32 <= N) {
+          float4 old[8];  // all loads before any store
+          if (keep) {
 #pragma unroll
-          for (int t = 0; t < 32; t += 4) {
-            float4 o = make_float4(v[t], v[t + 1], v[t + 2], v[t + 3]);
-            if (keep) {
-              const float4 old = *reinterpret_cast<const float4 *>(crow + t);
-              o.x += bw * old.x;
-              o.y += bw * old.y;
-              o.z += bw * old.z;
-              o.w += bw * old.w;
-            }
-            *reinterpret_cast<float4 *>(crow + t) = o;
+            for (int t = 0; t < 8; ++t) old[t] = __ldcg(reinterpret_cast<const float4 *>(crow) + t);
+          } else {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) old[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float4 o = make_float4(fmaf(bw, old[t].x, v[4 * t]),
+                                         fmaf(bw, old[t].y, v[4 * t + 1]),
+                                         fmaf(bw, old[t].z, v[4 * t + 2]),
+                                         fmaf(bw, old[t].w, v[4 * t + 3]));
+            reinterpret_cast<float4 *>(crow)[t] = o;
           }
         } else {
 #pragma unroll

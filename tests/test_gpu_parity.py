@@ -265,8 +265,8 @@ def test_gemm_f32_positive_long_k(cuda_device, split):
     Cholesky's Schur updates) over a long K: a one-way drift of the
     tensor-core accumulation (up to one unit in the last place per MMA step)
     adds up here instead of cancelling. The main accumulator restarts every
-    4096 k and the cross terms accumulate apart, so the drift stays below one
-    chunk's steps: (4096 / k-per-MMA) * 2^-23."""
+    8192 k and the cross terms accumulate apart, so the drift stays below one
+    chunk's steps: (8192 / k-per-MMA) * 2^-23."""
     Kq = K()
     M, N, Kd = 4096, 4096, 16384
     g = torch.Generator(device="cuda").manual_seed(7)
@@ -283,7 +283,7 @@ def test_gemm_f32_positive_long_k(cuda_device, split):
     want = a.double() @ a.double().T
     rel = float(((C.double() - want) / want).abs().max())
     kstep = 16 if split == "fp16" else 8
-    assert rel < (4096 // kstep) * 2.0 ** -23, rel
+    assert rel < (8192 // kstep) * 2.0 ** -23, rel
 
 
 @pytest.mark.parametrize("split", ["tf32", "fp16"])
