@@ -154,7 +154,8 @@ typedef enum {
   KRONQ_WS_BIIP = 0,
   KRONQ_WS_CHOL = 1,
   KRONQ_WS_QUANT = 2,
-  KRONQ_WS_LOSS = 3
+  KRONQ_WS_LOSS = 3,
+  KRONQ_WS_QUANT_SPLIT = 4
 } kronq_ws_kind;
 
 /*
@@ -293,6 +294,37 @@ kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,
 /* Workspace bytes that let kronq_gemm_f32 take the fp16 path (0 if M, N or
  * K <= 0). */
 size_t kronq_gemm_f32_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Steps 4 and 5 in split form (no counterpart on the pages: a cheaper route
+ * to the same OBS decisions). With H + λI = R Rᵀ (R upper) and U = R^-1,
+ * kronq_chol_split leaves
+ *     H = [U11, R12; 0, U22],  split at h = kronq_chol_split_point(d)
+ *                              = 128 * floor(d / 256),
+ * i.e. the root block right of the split keeps the Cholesky factor R12
+ * instead of the inverse factor U12, which saves the two products that form
+ * U12 (about d^3/4 flop of the 2 d^3/3). Same arguments, workspace
+ * (KRONQ_WS_CHOL) and errors as kronq_chol_inv; d >= 256.
+ *
+ * kronq_quantize_split runs the OBS sweep of kronq_quantize_sublayer on that
+ * form: the first h columns with U11, then the second half starting from
+ *     W2 + ((W1 - What1) R12) U22
+ * (the GPTQ recursion gives E U = W - What for the scaled errors E, so the
+ * first half reaches the second through R12 alone), with U22. The decisions
+ * are those of the one-pass sweep with the full U; the extra product costs
+ * d_out * m^2 flop (m = d_in - h), so the split pays when d_in > d_out.
+ * Arguments as kronq_quantize_sublayer with F the output of kronq_chol_split;
+ * workspace KRONQ_WS_QUANT_SPLIT; d_in >= 256.
+ */
+kronq_status kronq_chol_split(kronq_stream_t stream, float *H, int64_t d,
+                              float damp_rel, void *ws, size_t ws_bytes,
+                              int32_t *info_dev);
+int64_t kronq_chol_split_point(int64_t d);
+kronq_status kronq_quantize_split(kronq_stream_t stream, const kronq_opts *opts,
+                                  float *W_rot, const float *F, int64_t d_out,
+                                  int64_t d_in, uint32_t *codes, float *scales,
+                                  uint8_t *zeros, void *ws, size_t ws_bytes,
+                                  int32_t *info_dev);
 
 /* Workspace bytes needed by one call (opts may be NULL except for BIIP and
  * QUANT). Returns 0 for unsupported arguments. */

@@ -82,6 +82,9 @@ size_t kronq_workspace_bytes(kronq_ws_kind which, int64_t d_out, int64_t d_in,
       return quant_ws_bytes(d_out, d_in, *opts);
     case KRONQ_WS_LOSS:
       return loss_ws_bytes(d_out, d_in);
+    case KRONQ_WS_QUANT_SPLIT:
+      if (!opts || d_in % 128 || d_in < 256) return 0;
+      return quant_split_ws_bytes(d_out, d_in, chol_split_point(d_in), *opts);
   }
   return 0;
 }
@@ -149,6 +152,45 @@ kronq_status kronq_quantize_sublayer(kronq_stream_t stream,
   KQ_TRY(launch_set_int(st, info_dev, 0));
   return quantize(st, *opts, W_rot, U, d_out, d_in, codes, scales, zeros, ws,
                   ws_bytes, info_dev);
+}
+
+kronq_status kronq_chol_split(kronq_stream_t stream, float *H, int64_t d,
+                              float damp_rel, void *ws, size_t ws_bytes,
+                              int32_t *info_dev) {
+  if (!H || !ws || !info_dev || d <= 0 || !(damp_rel >= 0.f) || !isfinite(damp_rel))
+    return KRONQ_ERR_INVALID_ARG;
+  if (d % 128 || d < 256 || d > 65536) return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !aligned(H, 16)) return KRONQ_ERR_INVALID_ARG;
+  if (ws_bytes < chol_ws_bytes(d)) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return chol_split(st, H, d, damp_rel, ws, ws_bytes, info_dev);
+}
+
+int64_t kronq_chol_split_point(int64_t d) { return d >= 256 ? chol_split_point(d) : 0; }
+
+kronq_status kronq_quantize_split(kronq_stream_t stream, const kronq_opts *opts,
+                                  float *W_rot, const float *F, int64_t d_out,
+                                  int64_t d_in, uint32_t *codes, float *scales,
+                                  uint8_t *zeros, void *ws, size_t ws_bytes,
+                                  int32_t *info_dev) {
+  if (!opts || !W_rot || !F || !codes || !scales || !zeros || !ws || !info_dev ||
+      d_out <= 0 || d_in <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  if (opts->bits < 2 || opts->bits > 4) return KRONQ_ERR_INVALID_ARG;
+  if (opts->group != 32 && opts->group != 64 && opts->group != 128)
+    return KRONQ_ERR_UNSUPPORTED;
+  if (opts->block != 128 || d_in % 128 || d_in < 256) return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !aligned(W_rot, 16) || !aligned(F, 16))
+    return KRONQ_ERR_INVALID_ARG;
+  const int64_t h = chol_split_point(d_in);
+  if (ws_bytes < quant_split_ws_bytes(d_out, d_in, h, *opts)) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return quantize_split(st, *opts, W_rot, F, d_out, d_in, h, codes, scales, zeros, ws,
+                        ws_bytes, info_dev);
 }
 
 kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,

@@ -240,6 +240,7 @@ struct Ctx {
   size_t scr_main_bytes, scr_side_bytes[MAXD];
   const float *lambda;
   int32_t *info;
+  bool root_r;               // keep R12 at the root instead of U12 (no T, no U12)
 };
 
 // Streams and events of the recursion, created once per device: the critical
@@ -308,7 +309,9 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.kflags = KR_B_UPPER;
     KQ_TRY(gemm_f32(c.st, g, c.scr_main, c.scr_main_bytes, c.info));
   }
+  const bool keep_r = c.root_r && depth == 0;
   // T = V U22 does not feed the recursion into A11: run it beside it
+  if (!keep_r) {
   if (cudaEventRecord(c.ev_v[depth], c.st) != cudaSuccess ||
       cudaStreamWaitEvent(c.side[depth], c.ev_v[depth], 0) != cudaSuccess)
     return KRONQ_ERR_CUDA;
@@ -323,6 +326,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
   }
   if (cudaEventRecord(c.ev_t[depth], c.side[depth]) != cudaSuccess)
     return KRONQ_ERR_CUDA;
+  }
   {
     GemmArgs g;  // A11 -= V Vᵀ (tiles on or above the diagonal)
     g.M = h; g.N = h; g.K = m;
@@ -334,6 +338,13 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     KQ_TRY(gemm_f32(c.st, g, c.scr_main, c.scr_main_bytes, c.info));
   }
   KQ_TRY(rinv(c, off, h, depth + 1));  // A11 -> U11
+  if (keep_r) {
+    // the caller's OBS crosses the halves with R12 = V itself
+    if (cudaMemcpy2DAsync(B12, static_cast<size_t>(d) * 4, V, static_cast<size_t>(m) * 4,
+                          static_cast<size_t>(m) * 4, static_cast<size_t>(h),
+                          cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return KRONQ_ERR_CUDA;
+  } else {
   if (cudaStreamWaitEvent(c.st, c.ev_t[depth], 0) != cudaSuccess) return KRONQ_ERR_CUDA;
   {
     GemmArgs g;  // U12 = -U11 T : U11[i][k] == 0 for k < i
@@ -344,6 +355,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.alpha = -1.f;
     g.kflags = KR_A_UPPER;
     KQ_TRY(gemm_f32(c.st, g, c.scr_main, c.scr_main_bytes, c.info));
+  }
   }
   // zeros below the diagonal of this node (the leaves zero their own blocks):
   // triangular operands of the parents' products read U as 128 x 256 tiles
@@ -394,8 +406,8 @@ CholLayout chol_layout(int64_t d) {
 
 size_t chol_ws_bytes(int64_t d) { return chol_layout(d).total; }
 
-kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
-                      void *ws, size_t ws_bytes, int32_t *info) {
+kronq_status chol_run(cudaStream_t st, float *H, int64_t d, float damp_rel,
+                      void *ws, size_t ws_bytes, int32_t *info, bool root_r) {
   const CholLayout lay = chol_layout(d);
   const int depths = lay.depths;
   const size_t need = lay.total;
@@ -424,6 +436,7 @@ kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
   float *lambda = reinterpret_cast<float *>(w + need - 256);
   c.lambda = lambda;
   c.info = info;
+  c.root_r = root_r && d > NB;
   // fork from the caller's stream
   if (cudaEventRecord(cs->fork, st) != cudaSuccess ||
       cudaStreamWaitEvent(cs->main, cs->fork, 0) != cudaSuccess)
@@ -444,5 +457,17 @@ kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
       return KRONQ_ERR_CUDA;
   return KRONQ_OK;
 }
+
+kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
+                      void *ws, size_t ws_bytes, int32_t *info) {
+  return chol_run(st, H, d, damp_rel, ws, ws_bytes, info, false);
+}
+
+kronq_status chol_split(cudaStream_t st, float *H, int64_t d, float damp_rel,
+                        void *ws, size_t ws_bytes, int32_t *info) {
+  return chol_run(st, H, d, damp_rel, ws, ws_bytes, info, true);
+}
+
+int64_t chol_split_point(int64_t d) { return first_half(d); }
 
 }  // namespace kronq

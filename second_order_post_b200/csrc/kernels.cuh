@@ -60,6 +60,11 @@ uint64_t launches();
 size_t chol_ws_bytes(int64_t d);
 kronq_status chol_inv(cudaStream_t st, float *H, int64_t d, float damp_rel,
                       void *ws, size_t ws_bytes, int32_t *info);
+// Same recursion, but the root keeps R12 (= V) in place of U12:
+// H <- [U11, R12; 0, U22] split at chol_split_point(d).
+kronq_status chol_split(cudaStream_t st, float *H, int64_t d, float damp_rel,
+                        void *ws, size_t ws_bytes, int32_t *info);
+int64_t chol_split_point(int64_t d);
 
 // ---------------------------------------------------------------- BiIP
 size_t biip_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &o);
@@ -74,6 +79,25 @@ kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
                       const float *U, int64_t d_out, int64_t d_in,
                       uint32_t *codes, float *scales, uint8_t *zeros,
                       void *ws, size_t ws_bytes, int32_t *info);
+struct QuantView {
+  float *W;
+  int64_t ldw;
+  const float *U;
+  int64_t ldu;
+  uint32_t *codes;
+  int64_t ldq;       // words per row of the full code array
+  float *scales;
+  uint8_t *zeros;
+  int64_t lds;       // groups per row of the full scale / zero arrays
+  int64_t d_out, n;  // rows, columns of the view
+};
+kronq_status quantize_view(cudaStream_t st, const kronq_opts &o, const QuantView &v,
+                           void *ws, size_t ws_bytes, int32_t *info);
+size_t quant_split_ws_bytes(int64_t d_out, int64_t d_in, int64_t h, const kronq_opts &o);
+kronq_status quantize_split(cudaStream_t st, const kronq_opts &o, float *W,
+                            const float *F, int64_t d_out, int64_t d_in, int64_t h,
+                            uint32_t *codes, float *scales, uint8_t *zeros,
+                            void *ws, size_t ws_bytes, int32_t *info);
 
 // ---------------------------------------------------------------- loss
 size_t loss_ws_bytes(int64_t d_out, int64_t d_in);

@@ -174,6 +174,15 @@ __global__ void __launch_bounds__(OTHREADS)
   }
 }
 
+__global__ void diff_inplace_kernel(float *__restrict__ A, int64_t lda,
+                                    const float *__restrict__ B, int64_t ldb,
+                                    int64_t rows, int64_t cols) {
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y)
+    for (int64_t c = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; c < cols;
+         c += int64_t(gridDim.x) * blockDim.x)
+      A[r * lda + c] -= B[r * ldb + c];
+}
+
 }  // namespace
 
 // Workspace: the errors E (d_out x S), then scratch for the super-block
@@ -184,18 +193,18 @@ size_t quant_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &) {
   return e + gemm_scratch_bytes(d_out, d_in - S, S) + 256;
 }
 
-kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
-                      const float *U, int64_t d_out, int64_t d_in,
-                      uint32_t *codes, float *scales, uint8_t *zeros,
-                      void *ws, size_t ws_bytes, int32_t *info) {
-  if (ws_bytes < quant_ws_bytes(d_out, d_in, o)) return KRONQ_ERR_INVALID_ARG;
-  const int64_t S = kq_min<int64_t>(d_in, SUPER);
+// OBS over the n columns of a strided view: W (pitch ldw), its U block
+// (pitch ldu), and the codes / scales / zeros of those columns (row pitches
+// ldq words and lds groups of the full arrays).
+kronq_status quantize_view(cudaStream_t st, const kronq_opts &o, const QuantView &v,
+                           void *ws, size_t ws_bytes, int32_t *info) {
+  const int64_t d_out = v.d_out, n = v.n;
+  if (ws_bytes < quant_ws_bytes(d_out, n, o)) return KRONQ_ERR_INVALID_ARG;
+  const int64_t S = kq_min<int64_t>(n, SUPER);
   float *E = static_cast<float *>(ws);
   const size_t e_bytes = (static_cast<size_t>(d_out) * S * 4 + 255) / 256 * 256;
   void *scr = static_cast<uint8_t *>(ws) + e_bytes;
   const size_t scr_bytes = ws_bytes - e_bytes;
-  const int64_t ngroups = d_in / o.group;
-  const int64_t ldq = o.bits * d_in / 32;
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(obs_block_kernel,
@@ -204,35 +213,115 @@ kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
       return KRONQ_ERR_CUDA;
     attr_done = true;
   }
+  float *W = v.W;
+  const float *U = v.U;
   const unsigned grid = static_cast<unsigned>(ceil_div(d_out, OROWS));
-  for (int64_t sb0 = 0; sb0 < d_in; sb0 += S) {
-    const int64_t sb1 = kq_min<int64_t>(d_in, sb0 + S);
+  for (int64_t sb0 = 0; sb0 < n; sb0 += S) {
+    const int64_t sb1 = kq_min<int64_t>(n, sb0 + S);
     for (int64_t j0 = sb0; j0 < sb1; j0 += OB) {
       obs_block_kernel<<<grid, OTHREADS, OSMEM, st>>>(
-          W, d_in, U, d_in, j0, d_out, o.bits, o.group, E, S, j0 - sb0, codes,
-          ldq, scales, zeros, ngroups);
+          W, v.ldw, U, v.ldu, j0, d_out, o.bits, o.group, E, S, j0 - sb0, v.codes,
+          v.ldq, v.scales, v.zeros, v.lds);
       KQ_CHECK_LAUNCH();
       if (j0 + OB < sb1) {
         GemmArgs g;
         g.M = d_out; g.N = sb1 - j0 - OB; g.K = OB;
         g.A = E + (j0 - sb0); g.lda = S;
-        g.B = U + j0 * d_in + j0 + OB; g.ldb = d_in; g.b_mn = true;
-        g.C = W + j0 + OB; g.ldc = d_in;
+        g.B = U + j0 * v.ldu + j0 + OB; g.ldb = v.ldu; g.b_mn = true;
+        g.C = W + j0 + OB; g.ldc = v.ldw;
         g.alpha = -1.f; g.beta = 1.f;
         KQ_TRY(gemm_tf32x3(st, g, info));
       }
     }
-    if (sb1 < d_in) {
+    if (sb1 < n) {
       GemmArgs g;
-      g.M = d_out; g.N = d_in - sb1; g.K = sb1 - sb0;
+      g.M = d_out; g.N = n - sb1; g.K = sb1 - sb0;
       g.A = E; g.lda = S;
-      g.B = U + sb0 * d_in + sb1; g.ldb = d_in; g.b_mn = true;
-      g.C = W + sb1; g.ldc = d_in;
+      g.B = U + sb0 * v.ldu + sb1; g.ldb = v.ldu; g.b_mn = true;
+      g.C = W + sb1; g.ldc = v.ldw;
       g.alpha = -1.f; g.beta = 1.f;
       KQ_TRY(gemm_f32(st, g, scr, scr_bytes, info));
     }
   }
   return KRONQ_OK;
+}
+
+kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
+                      const float *U, int64_t d_out, int64_t d_in,
+                      uint32_t *codes, float *scales, uint8_t *zeros,
+                      void *ws, size_t ws_bytes, int32_t *info) {
+  QuantView v{W, d_in, U, d_in, codes, o.bits * d_in / 32, scales, zeros,
+              d_in / o.group, d_out, d_in};
+  return quantize_view(st, o, v, ws, ws_bytes, info);
+}
+
+// ---------------------------------------------------------------- split form
+// OBS on the output of chol_split, F = [U11, R12; 0, U22] (H + λI = R Rᵀ with
+// R upper, U = R^-1, split at h). The sweep over the first h columns uses
+// U11. Its results enter the second half through R12 alone: the GPTQ
+// recursion gives E·U = W − Ŵ for the scaled errors E, so E = (W − Ŵ)·R,
+// and the second half starts from
+//     W2 + ((W1 − Ŵ1) R12) U22,
+// after which the sweep over the second half uses U22. The result equals the
+// one-pass sweep with the full U (same decisions; the products differ by
+// rounding).
+size_t quant_split_ws_bytes(int64_t d_out, int64_t d_in, int64_t h, const kronq_opts &o) {
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  const int64_t m = d_in - h;
+  const size_t save = al(static_cast<size_t>(d_out) * h * 4);
+  const size_t p = al(static_cast<size_t>(d_out) * m * 4);
+  const size_t sweep = kq_max(quant_ws_bytes(d_out, h, o), quant_ws_bytes(d_out, m, o));
+  const size_t cross = kq_max(gemm_scratch_bytes(d_out, m, h), gemm_scratch_bytes(d_out, m, m));
+  return save + p + kq_max(sweep, cross) + 256;
+}
+
+kronq_status quantize_split(cudaStream_t st, const kronq_opts &o, float *W,
+                            const float *F, int64_t d_out, int64_t d_in, int64_t h,
+                            uint32_t *codes, float *scales, uint8_t *zeros,
+                            void *ws, size_t ws_bytes, int32_t *info) {
+  if (ws_bytes < quant_split_ws_bytes(d_out, d_in, h, o)) return KRONQ_ERR_INVALID_ARG;
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  const int64_t m = d_in - h;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  float *W1 = reinterpret_cast<float *>(w);               // W1, then W1 − Ŵ1
+  w += al(static_cast<size_t>(d_out) * h * 4);
+  float *P = reinterpret_cast<float *>(w);                // (W1 − Ŵ1) R12
+  w += al(static_cast<size_t>(d_out) * m * 4);
+  const size_t rest = ws_bytes - (static_cast<size_t>(w - static_cast<uint8_t *>(ws)));
+  const int64_t ldq = o.bits * d_in / 32, lds = d_in / o.group;
+  if (cudaMemcpy2DAsync(W1, static_cast<size_t>(h) * 4, W, static_cast<size_t>(d_in) * 4,
+                        static_cast<size_t>(h) * 4, static_cast<size_t>(d_out),
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return KRONQ_ERR_CUDA;
+  QuantView v1{W, d_in, F, d_in, codes, ldq, scales, zeros, lds, d_out, h};
+  KQ_TRY(quantize_view(st, o, v1, w, rest, info));
+  {  // W1 − Ŵ1
+    dim3 grid(static_cast<unsigned>(kq_min<int64_t>(ceil_div(h, 256), 16)),
+              static_cast<unsigned>(kq_min<int64_t>(d_out, 65535)));
+    diff_inplace_kernel<<<grid, 256, 0, st>>>(W1, h, W, d_in, d_out, h);
+    KQ_CHECK_LAUNCH();
+  }
+  {
+    GemmArgs g;  // P = (W1 − Ŵ1) R12
+    g.M = d_out; g.N = m; g.K = h;
+    g.A = W1; g.lda = h;
+    g.B = F + h; g.ldb = d_in; g.b_mn = true;
+    g.C = P; g.ldc = m;
+    KQ_TRY(gemm_f32(st, g, w, rest, info));
+  }
+  {
+    GemmArgs g;  // W2 += P U22 : U22[k][j] == 0 for k > j
+    g.M = d_out; g.N = m; g.K = m;
+    g.A = P; g.lda = m;
+    g.B = F + h * d_in + h; g.ldb = d_in; g.b_mn = true;
+    g.C = W + h; g.ldc = d_in;
+    g.beta = 1.f;
+    g.kflags = KR_B_LOWER;
+    KQ_TRY(gemm_f32(st, g, w, rest, info));
+  }
+  QuantView v2{W + h, d_in, F + h * d_in + h, d_in, codes + o.bits * h / 32, ldq,
+               scales + h / o.group, zeros + h / o.group, lds, d_out, m};
+  return quantize_view(st, o, v2, w, rest, info);
 }
 
 }  // namespace kronq

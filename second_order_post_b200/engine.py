@@ -9,6 +9,9 @@ across calls) and enqueues the five steps on one CUDA stream:
   4. kronq_chol_inv(H_X') -> U               (in place)
   5. kronq_quantize_sublayer(W', U) -> codes, scales, zeros, W_hat (in place)
 
+When d_in > d_out, steps 4 and 5 take the split form (kronq_chol_split,
+kronq_quantize_split): the same OBS decisions for fewer flops.
+
 All arithmetic runs in the library's kernels; this module only allocates and
 passes pointers.
 """
@@ -35,8 +38,11 @@ class QuantResult:
 class SublayerEngine:
     def __init__(self, d_out, d_in, bits=4, group=128, damp_rel=0.01,
                  scale_exp=0.25, seed=0, rot_in=None, rot_out=None, flags=0,
-                 device="cuda", keep_w_rot=False):
+                 device="cuda", keep_w_rot=False, split=None):
         self.d_out, self.d_in = d_out, d_in
+        # the split form saves d^3/4 flop in the Cholesky step and spends
+        # d_out * (d_in/2)^2 more in the OBS step: worth it when d_in > d_out
+        self.split = (d_in > d_out and d_in >= 256) if split is None else split
         self.opts = K.make_opts(bits=bits, group=group, damp_rel=damp_rel,
                                 scale_exp=scale_exp, seed=seed,
                                 rot_in=rot_in or (d_in, 1),
@@ -55,9 +61,9 @@ class SublayerEngine:
         self.scales = torch.empty(d_out, ng, **f32)
         self.zeros = torch.empty(d_out, ng, dtype=torch.uint8, device=dev)
         self.info = torch.zeros(3, dtype=torch.int32, device=dev)
-        ws = max(K.kronq_workspace_bytes(K.KRONQ_WS_BIIP, d_out, d_in, self.opts),
-                 K.kronq_workspace_bytes(K.KRONQ_WS_CHOL, d_out, d_in, self.opts),
-                 K.kronq_workspace_bytes(K.KRONQ_WS_QUANT, d_out, d_in, self.opts))
+        kinds = [K.KRONQ_WS_BIIP, K.KRONQ_WS_CHOL,
+                 K.KRONQ_WS_QUANT_SPLIT if self.split else K.KRONQ_WS_QUANT]
+        ws = max(K.kronq_workspace_bytes(k, d_out, d_in, self.opts) for k in kinds)
         if ws == 0:
             raise ValueError("unsupported sublayer shape for libkronq")
         self.ws = torch.empty((ws + 255) // 256 * 256, dtype=torch.uint8, device=dev)
@@ -81,12 +87,20 @@ class SublayerEngine:
         mark("biip")
         if self.W_ref is not None:
             self.W_ref.copy_(self.W_rot)
-        K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[1:2],
-                         stream)
-        mark("chol")
-        K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, self.codes,
-                                  self.scales, self.zeros, self.ws,
-                                  self.info[2:3], stream)
+        if self.split:
+            K.kronq_chol_split(self.H_X, self.opts.damp_rel, self.ws,
+                               self.info[1:2], stream)
+            mark("chol")
+            K.kronq_quantize_split(self.opts, self.W_rot, self.H_X, self.codes,
+                                   self.scales, self.zeros, self.ws,
+                                   self.info[2:3], stream)
+        else:
+            K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[1:2],
+                             stream)
+            mark("chol")
+            K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, self.codes,
+                                      self.scales, self.zeros, self.ws,
+                                      self.info[2:3], stream)
         mark("quant")
         return QuantResult(self.codes, self.scales, self.zeros, self.W_rot,
                            self.s_x, self.s_g, self.sens)
@@ -94,7 +108,9 @@ class SublayerEngine:
     def check_info(self):
         """Raises KronqError for a non-zero device status word (syncs)."""
         vals = self.info.tolist()
-        for name, v in zip(("kronq_biip", "kronq_chol_inv",
-                            "kronq_quantize_sublayer"), vals):
+        names = (("kronq_biip", "kronq_chol_split", "kronq_quantize_split")
+                 if self.split else
+                 ("kronq_biip", "kronq_chol_inv", "kronq_quantize_sublayer"))
+        for name, v in zip(names, vals):
             if v != 0:
                 raise K.KronqError(name, v & 0xFF)

@@ -36,7 +36,7 @@ KRONQ_BF16 = 1
 KRONQ_FLAG_NO_ROT_IN = 0x1
 KRONQ_FLAG_NO_ROT_OUT = 0x2
 KRONQ_FLAG_NO_SCALE = 0x4
-KRONQ_WS_BIIP, KRONQ_WS_CHOL, KRONQ_WS_QUANT, KRONQ_WS_LOSS = 0, 1, 2, 3
+KRONQ_WS_BIIP, KRONQ_WS_CHOL, KRONQ_WS_QUANT, KRONQ_WS_LOSS, KRONQ_WS_QUANT_SPLIT = 0, 1, 2, 3, 4
 
 
 class kronq_rot(ctypes.Structure):
@@ -78,6 +78,9 @@ _SIGS = {
     "kronq_quantize_sublayer": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p,
                                 _sz, _p],
     "kronq_layer_loss": [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _sz],
+    "kronq_chol_split": [_p, _p, _i64, _f, _p, _sz, _p],
+    "kronq_chol_split_point": [_i64],
+    "kronq_quantize_split": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p, _sz, _p],
     "kronq_gemm_f32": [_p, _i64, _i64, _i64, _f, _p, _i64, ctypes.c_int, _p,
                        _i64, ctypes.c_int, _f, _p, _i64, _p, _sz, _p],
     "kronq_gemm_f32_workspace_bytes": [_i64, _i64, _i64],
@@ -92,6 +95,7 @@ for _name, _args in _SIGS.items():
     _fn.restype = ctypes.c_int
 _lib.kronq_workspace_bytes.restype = ctypes.c_size_t
 _lib.kronq_gemm_f32_workspace_bytes.restype = ctypes.c_size_t
+_lib.kronq_chol_split_point.restype = ctypes.c_int64
 _lib.kronq_status_string.restype = ctypes.c_char_p
 _lib.kronq_kernel_launches.restype = ctypes.c_uint64
 
@@ -169,6 +173,25 @@ def kronq_quantize_sublayer(opts, W_rot, U, codes, scales, zeros, ws, info,
     d_out, d_in = W_rot.shape
     _check("kronq_quantize_sublayer", _lib.kronq_quantize_sublayer(
         _stream(stream), ctypes.byref(opts), _ptr(W_rot), _ptr(U), d_out, d_in,
+        _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(info)))
+
+
+def kronq_chol_split(H, damp_rel, ws, info, stream=None):
+    _check("kronq_chol_split", _lib.kronq_chol_split(
+        _stream(stream), _ptr(H), H.shape[0], damp_rel, _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(info)))
+
+
+def kronq_chol_split_point(d):
+    return _lib.kronq_chol_split_point(d)
+
+
+def kronq_quantize_split(opts, W_rot, F, codes, scales, zeros, ws, info,
+                         stream=None):
+    d_out, d_in = W_rot.shape
+    _check("kronq_quantize_split", _lib.kronq_quantize_split(
+        _stream(stream), ctypes.byref(opts), _ptr(W_rot), _ptr(F), d_out, d_in,
         _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(info)))
 

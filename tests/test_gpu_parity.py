@@ -251,6 +251,53 @@ def test_quantize_sampled_rows(cuda_device):
     assert ident >= 0.999
 
 
+# split form: kronq_chol_split + kronq_quantize_split against the one-pass OBS
+@pytest.mark.parametrize("d_out,d_in,bits,group", [
+    (128, 1024, 2, 128), (96, 1152, 3, 64), (64, 640, 4, 32)])
+def test_split_form(cuda_device, d_out, d_in, bits, group):
+    Kq = K()
+    data = synth.small_case(d_out, d_in, 2 * d_in, seed=d_in + 7 * bits)
+    w32 = data["W"].numpy().astype(np.float32)
+    hx = O.cov(data["X"].numpy())
+    F = dev(hx.astype(np.float32))
+    ws = torch.empty(Kq.kronq_workspace_bytes(Kq.KRONQ_WS_CHOL, d_out, d_in),
+                     dtype=torch.uint8, device="cuda")
+    info = torch.ones(1, dtype=torch.int32, device="cuda")
+    Kq.kronq_chol_split(F, 0.01, ws, info)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    h = Kq.kronq_chol_split_point(d_in)
+    assert h == (d_in // 256) * 128
+    # the three blocks against the oracle's U and R = U^-1
+    u = O.chol_inv(hx, 0.01)
+    r = np.linalg.inv(u)
+    f = f64(F)
+    assert rel_fro(f[:h, :h], u[:h, :h]) < 2e-4
+    assert rel_fro(f[h:, h:], u[h:, h:]) < 2e-4
+    assert rel_fro(f[:h, h:], r[:h, h:]) < 2e-4
+    assert np.count_nonzero(np.tril(f, -1)) == 0
+    opts = Kq.make_opts(bits=bits, group=group)
+    W = dev(w32)
+    codes = torch.empty(d_out, bits * d_in // 32, dtype=torch.int32, device="cuda")
+    scales = torch.empty(d_out, d_in // group, device="cuda")
+    zeros = torch.empty(d_out, d_in // group, dtype=torch.uint8, device="cuda")
+    qws = torch.empty(Kq.kronq_workspace_bytes(Kq.KRONQ_WS_QUANT_SPLIT, d_out, d_in, opts),
+                      dtype=torch.uint8, device="cuda")
+    Kq.kronq_quantize_split(opts, W, F, codes, scales, zeros, qws, info)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    got_codes = O.unpack_codes(codes.cpu().numpy().view(np.uint32), bits, d_in)
+    got_zeros = zeros.cpu().numpy().astype(np.int64)
+    w64 = w32.astype(np.float64)
+    ref = O.obs_quantize(w64, u, bits, group)
+    assert (got_codes == ref["codes"]).mean() >= 0.999
+    ident, n_bad, _ = replay_check(w64, u, got_codes, got_zeros, bits, group)
+    assert n_bad == 0
+    assert ident >= 0.999
+    rep = O.obs_quantize(w64, u, bits, group, forced_codes=got_codes, forced_zeros=got_zeros)
+    assert rel_fro(f64(W), rep["w_hat"]) < 1e-5
+
+
 # ------------------------------------------------------------------ GEMM
 # (M, N, K, a_mn, b_mn): narrow 128 x 128 tiles, ragged edges, and the wide
 # 128 x 256 tiles in every operand major

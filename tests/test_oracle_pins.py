@@ -360,3 +360,27 @@ def test_layer_loss_is_kronecker_quadratic_form():
 ])
 def test_allocator_hand(scores, numel, budget, want):
     assert O.allocate_bits(scores, numel, budget) == want
+
+
+def test_obs_two_halves_join_through_r12():
+    """The GPTQ recursion gives E U = W - W_hat for the scaled errors E, so
+    E = (W - W_hat) R with R = U^-1 (H + lambda I = R R^T): the sweep over the
+    first h columns reaches the rest only through R12, and running the second
+    half from W2 + ((W1 - W_hat1) R12) U22 with U22 reproduces the one-pass
+    sweep (same codes, same dequantized weights)."""
+    rng = np.random.default_rng(21)
+    d_out, d_in, h = 24, 96, 40
+    x = rng.standard_normal((3 * d_in, d_in)) @ (np.eye(d_in) + 0.3 * rng.standard_normal((d_in, d_in)) / np.sqrt(d_in))
+    x *= np.exp(rng.uniform(-1, 1, d_in))
+    hx = x.T @ x / x.shape[0]
+    w = rng.standard_normal((d_out, d_in)) * 0.02
+    u = O.chol_inv(hx, 0.01)
+    r = np.linalg.inv(u)
+    for bits, group in ((2, 8), (3, 4), (4, 8)):
+        whole = O.obs_quantize(w, u, bits, group)
+        first = O.obs_quantize(w[:, :h], u[:h, :h], bits, group)
+        w2 = w[:, h:] + ((w[:, :h] - first["w_hat"]) @ r[:h, h:]) @ u[h:, h:]
+        second = O.obs_quantize(w2, u[h:, h:], bits, group)
+        assert np.array_equal(np.concatenate([first["codes"], second["codes"]], 1), whole["codes"])
+        assert np.allclose(np.concatenate([first["w_hat"], second["w_hat"]], 1), whole["w_hat"],
+                           atol=1e-12)

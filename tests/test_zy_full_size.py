@@ -14,8 +14,11 @@ outputs it computes one by one or properties that hold at any size:
                u_i^T (S M S) u_j with rows u of the rotations built by the
                oracle from the published construction
   U            sampled columns of U^T U (H' + lambda I) against the identity
+               (per block in the split form [U11, R12; 0, U22] the engine
+               takes for d_in > d_out)
   codes        sampled rows replayed through the oracle's OBS sweep given the
-               device's U (rows are independent given U)
+               device's factor (rows are independent given U; in the split
+               form, two half sweeps joined through R12)
 """
 import math
 
@@ -64,9 +67,14 @@ def run(cuda_device):
     K.kronq_biip(eng.opts, W, eng.W_rot, eng.H_X, eng.H_G, eng.s_x, eng.s_g,
                  eng.ws, eng.info[0:1])
     HX1, W1 = eng.H_X.clone(), eng.W_rot.clone()
-    K.kronq_chol_inv(eng.H_X, wl.damp_rel, eng.ws, eng.info[1:2])
-    K.kronq_quantize_sublayer(eng.opts, eng.W_rot, eng.H_X, eng.codes, eng.scales,
-                              eng.zeros, eng.ws, eng.info[2:3])
+    if eng.split:   # the engine's choice for this shape (d_in > d_out)
+        K.kronq_chol_split(eng.H_X, wl.damp_rel, eng.ws, eng.info[1:2])
+        K.kronq_quantize_split(eng.opts, eng.W_rot, eng.H_X, eng.codes, eng.scales,
+                               eng.zeros, eng.ws, eng.info[2:3])
+    else:
+        K.kronq_chol_inv(eng.H_X, wl.damp_rel, eng.ws, eng.info[1:2])
+        K.kronq_quantize_sublayer(eng.opts, eng.W_rot, eng.H_X, eng.codes, eng.scales,
+                                  eng.zeros, eng.ws, eng.info[2:3])
     torch.cuda.synchronize()
     eng.check_info()
     return dict(wl=wl, W=W, X=X, G=G, eng=eng, HX0=HX0, HG0=HG0, HX1=HX1, W1=W1)
@@ -152,36 +160,94 @@ def test_biip_sampled_entries(run):
             assert abs(float(HX1[i, j]) - want) <= 1e-5 * scale
 
 
-def test_inverse_factor_residual(run):
-    """Columns of U^T U (H' + lambda I) - I at sampled positions; U comes from
-    fp32 arithmetic, so the bound is a few units of d * cond * 2^-24."""
-    wl, eng, HX1 = run["wl"], run["eng"], run["HX1"]
-    U = eng.H_X
+def _inverse_factor_residual(U, Hc, lam, cols, extra=None):
+    """max |U^T U (Hc + lambda I) - I| over the sampled columns (U upper,
+    Hc symmetric, both fp32 on the device); `extra(c, j)` may modify the
+    column of Hc + lambda I first."""
     d = U.shape[0]
-    assert int(torch.count_nonzero(torch.tril(U[:4096, :4096], -1))) == 0
-    lam = wl.damp_rel * float(torch.diag(HX1).double().mean())
-    rng = np.random.default_rng(3)
     worst = 0.0
-    for j in rng.choice(d, 6, replace=False):
-        c = HX1[:, int(j)].double().clone()
+    for j in cols:
+        c = Hc[:, int(j)].double().clone()
         c[int(j)] += lam
+        if extra is not None:
+            c = extra(c, int(j))
         y = _rows_matvec(U, c)                       # U c
         z = torch.zeros(d, dtype=torch.float64, device="cuda")
         for r0 in range(0, d, 2048):                 # U^T y
             z += U[r0:r0 + 2048].double().T @ y[r0:r0 + 2048]
         z[int(j)] -= 1.0
         worst = max(worst, float(z.abs().max()))
-    assert worst < 2e-3, worst
+    return worst
+
+
+def test_inverse_factor_residual(run):
+    """U^T U (H' + lambda I) - I on sampled columns; U comes from fp32
+    arithmetic, so the bound is a few units of d * cond * 2^-24. In the split
+    form [U11, R12; 0, U22] the checks are per block: U22 against the lower
+    right block C, U11 against the Schur complement A - R12 R12^T, and
+    R12 = B U22^T on sampled rows."""
+    wl, eng, HX1 = run["wl"], run["eng"], run["HX1"]
+    F = eng.H_X
+    d = F.shape[0]
+    assert int(torch.count_nonzero(torch.tril(F[:4096, :4096], -1))) == 0
+    lam = wl.damp_rel * float(torch.diag(HX1).double().mean())
+    rng = np.random.default_rng(3)
+    if not eng.split:
+        worst = _inverse_factor_residual(F, HX1, lam, rng.choice(d, 6, replace=False))
+        assert worst < 2e-3, worst
+        return
+    from second_order_post_b200 import kronq as K
+    h = K.kronq_chol_split_point(d)
+    U11, R12, U22 = F[:h, :h], F[:h, h:], F[h:, h:]
+    worst22 = _inverse_factor_residual(U22.contiguous(), HX1[h:, h:].contiguous(), lam,
+                                       rng.choice(d - h, 4, replace=False))
+    R12c = R12.contiguous()
+
+    def schur(c, j):   # column j of A + lambda I - R12 R12^T
+        return c - _rows_matvec(R12c, R12c[j].double())
+    worst11 = _inverse_factor_residual(U11.contiguous(), HX1[:h, :h].contiguous(), lam,
+                                       rng.choice(h, 4, replace=False), schur)
+    assert worst22 < 2e-3, worst22
+    assert worst11 < 2e-3, worst11
+    U22c = U22.contiguous()
+    for i in rng.choice(h, 4, replace=False):       # R12[i] = U22 B[i]^T
+        want = _rows_matvec(U22c, HX1[int(i), h:].double())
+        got = R12c[int(i)].double()
+        assert float((got - want).abs().max()) <= 1e-4 * float(want.abs().max())
 
 
 def test_codes_sampled_rows(run):
+    """Sampled rows replayed through the oracle's OBS sweep given the device's
+    factor. In the split form the replay runs in two halves joined through
+    R12 (W2 + ((W1 - W_hat1) R12) U22), which the oracle pins show equal to
+    the one-pass sweep."""
     wl, eng = run["wl"], run["eng"]
     rows = np.random.default_rng(4).choice(wl.d_out, 6, replace=False)
     ridx = torch.as_tensor(rows, device="cuda")
     w64 = run["W1"][ridx].double().cpu().numpy()
-    u64 = eng.H_X.double().cpu().numpy()
     codes = O.unpack_codes(eng.codes[ridx].cpu().numpy().view(np.uint32), wl.bits, wl.d_in)
     zeros = eng.zeros[ridx].cpu().numpy().astype(np.int64)
-    ident, n_bad, _ = replay_check(w64, u64, codes, zeros, wl.bits, wl.group)
-    assert n_bad == 0
-    assert ident >= 0.999
+    if not eng.split:
+        u64 = eng.H_X.double().cpu().numpy()
+        ident, n_bad, _ = replay_check(w64, u64, codes, zeros, wl.bits, wl.group)
+        assert n_bad == 0
+        assert ident >= 0.999
+        return
+    from second_order_post_b200 import kronq as K
+    h = K.kronq_chol_split_point(wl.d_in)
+    gh = h // wl.group
+    F = eng.H_X
+    u11 = F[:h, :h].double().cpu().numpy()
+    ident1, bad1, _ = replay_check(w64[:, :h], u11, codes[:, :h], zeros[:, :gh],
+                                   wl.bits, wl.group)
+    first = O.obs_quantize(w64[:, :h], u11, wl.bits, wl.group,
+                           forced_codes=codes[:, :h], forced_zeros=zeros[:, :gh])
+    del u11
+    r12 = F[:h, h:].double().cpu().numpy()
+    p = (w64[:, :h] - first["w_hat"]) @ r12
+    del r12
+    u22 = F[h:, h:].double().cpu().numpy()
+    w2 = w64[:, h:] + p @ u22
+    ident2, bad2, _ = replay_check(w2, u22, codes[:, h:], zeros[:, gh:], wl.bits, wl.group)
+    assert bad1 == 0 and bad2 == 0
+    assert min(ident1, ident2) >= 0.999
