@@ -3,175 +3,190 @@
 // and H_G does not enter it, so rows are independent given U; wmrh §五:
 // W2/W3/W4 with 128-column groups].
 //
-// Per 128-column block j0 (one launch of obs_block_kernel): each warp owns one
-// row at a time, the block's 128 weights of the row live in 4 registers per
-// lane, U[j0:j0+128, j0:j0+128] sits in shared memory. For each column j:
-// group (scale, zero) at a group start, q = clamp(rint(w/scale)+zero),
-// err = (w - w_hat)/U[j][j], w_k -= err * U[j][k] for the block's k > j.
-// The errors go to E; the columns right of the block are updated lazily by
-// 3xTF32 GEMMs: within a super-block of S columns after every block
-// (W[:, blk_end:sb_end] -= E_blk U[blk, blk_end:sb_end]), and once per
-// super-block for everything right of it (W[:, sb_end:] -= E_sb U[sb, sb_end:]).
-// Codes are packed in the same pass (little-endian bitstream per row).
+// Per 128-column block j0 (one launch of obs_block_kernel): four lanes share
+// one row, lane p of the quad holding the columns 4i + p (i < 32) in
+// registers, so that every lane has about the same number of updates left at
+// any column. U[j0:j0+128, j0:j0+128] sits in shared memory, permuted so that
+// each lane's columns of a U row are contiguous. The sweep over the block's
+// 128 columns is unrolled, so every register index is a compile-time
+// constant. For each column j: group (scale, zero) at a group start,
+// q = clamp(rint(w/scale)+zero), err = (w - w_hat)/U[j][j] (all four lanes
+// of the quad compute them from the owner's weight), w_k -= err * U[j][k] for
+// the block's k > j. The errors go to E; the columns right of the block are
+// updated lazily by 3xTF32 GEMMs: within a super-block of S columns after
+// every block (W[:, blk_end:sb_end] -= E_blk U[blk, blk_end:sb_end]), and
+// once per super-block for everything right of it
+// (W[:, sb_end:] -= E_sb U[sb, sb_end:]). Codes are packed in registers
+// during the sweep (little-endian bitstream per row).
+#include <utility>
+
 #include "kernels.cuh"
 
 namespace kronq {
 namespace {
 
-constexpr int OB = 128;        // block width
-constexpr int OTHREADS = 256;  // 8 warps
-constexpr int RPW = 4;         // rows per warp, swept together
-constexpr int OROWS = (OTHREADS / 32) * RPW;
-constexpr int SUPER = 1024;    // super-block width
-constexpr int OSMEM = (OB * OB + OB) * 4;
+constexpr int OB = 128;                    // block width
+constexpr int QLPR = 4;                    // lanes per row
+constexpr int QNI = OB / QLPR;             // columns (registers) per lane
+constexpr int QWARPS = 4;
+constexpr int OTHREADS = 32 * QWARPS;
+constexpr int OROWS = QWARPS * (32 / QLPR);  // rows per CTA
+constexpr int QUP = QNI + 4;               // one lane's run of a U row (padded)
+constexpr int QUROW = QLPR * QUP;          // floats per permuted U row
+constexpr int OSMEM = (OB * QUROW + OB) * 4;
+constexpr int SUPER = 1024;                // super-block width
 
-// Columns [32*SLOT, 32*SLOT + 32) of the block for the warp's RPW rows. With
-// the register slot fixed at compile time, columns left of the chunk need no
-// update and columns right of it are updated without predicates.
-template <int SLOT>
-__device__ __forceinline__ void obs_chunk(float (&w)[RPW][4], float (&err)[RPW][4],
-                                          float (&scale)[RPW], float (&rscale)[RPW],
-                                          float (&zero)[RPW], const float *Us,
-                                          const float *inv, uint8_t (*qs)[OB],
-                                          int lane, int group, float maxq,
-                                          int64_t row0, int64_t d_out, int64_t j0,
-                                          float *scales, uint8_t *zeros,
-                                          int64_t ngroups) {
-  constexpr int jb = 32 * SLOT;
-  if (jb % group == 0) {
-    // group start: (scale, zero) from the rows' current weights of the group
-    float mn[RPW], mx[RPW];
+// State of one lane during the sweep of a block.
+template <int BITS>
+struct SweepState {
+  static constexpr int NW = OB * BITS / 32;  // code words of the block per row
+  float w[QNI], err[QNI];
+  uint32_t cw[NW];
+  float scale, rscale, zero;
+};
+
+// Where a row's group parameters go: scales[gi], zeros[gi] for the group gi
+// that starts at block column J is gi = g0 + J / group.
+struct GroupOut {
+  float *scales;
+  uint8_t *zeros;
+  int64_t g0;
+  bool store;
+};
+
+// Column J of the block (every register index is a compile-time constant).
+template <int BITS, int J>
+__device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
+                                           const float *inv, int p, int quad,
+                                           int group, const GroupOut &go) {
+  constexpr int io = J / QLPR, po = J % QLPR;
+  constexpr float maxq = static_cast<float>((1 << BITS) - 1);
+  if constexpr (J % 32 == 0) {
+    if (J % group == 0) {
+      // group start: (scale, zero) from the row's current weights of the group
+      float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      mn[r] = INFINITY;
-      mx[r] = -INFINITY;
-#pragma unroll
-      for (int s = SLOT; s < 4; ++s) {
-        if (32 * s < jb + group) {
-          mn[r] = fminf(mn[r], w[r][s]);
-          mx[r] = fmaxf(mx[r], w[r][s]);
+      for (int i = io; i < QNI; ++i) {
+        if (QLPR * i < J + group) {
+          mn = fminf(mn, S.w[i]);
+          mx = fmaxf(mx, S.w[i]);
         }
       }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
+      for (int o = 1; o < QLPR; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float xmin = fminf(mn[r], 0.f), xmax = fmaxf(mx[r], 0.f);
+      const float xmin = fminf(mn, 0.f), xmax = fmaxf(mx, 0.f);
       if (xmax == xmin) {
-        scale[r] = 1.f;
-        zero[r] = 0.f;
+        S.scale = 1.f;
+        S.zero = 0.f;
       } else {
-        scale[r] = (xmax - xmin) / maxq;
-        zero[r] = rintf(-xmin / scale[r]);
+        S.scale = (xmax - xmin) / maxq;
+        S.zero = rintf(-xmin / S.scale);
       }
-      rscale[r] = 1.f / scale[r];
-      if (lane == 0 && row0 + r < d_out) {
-        const int64_t gi = (j0 + jb) / group;
-        scales[(row0 + r) * ngroups + gi] = scale[r];
-        zeros[(row0 + r) * ngroups + gi] = static_cast<uint8_t>(zero[r]);
+      S.rscale = 1.f / S.scale;
+      if (go.store) {
+        const int64_t gi = go.g0 + J / group;
+        go.scales[gi] = S.scale;
+        go.zeros[gi] = static_cast<uint8_t>(S.zero);
       }
     }
   }
-  for (int jj = 0; jj < 32; ++jj) {
-    const int j = jb + jj;
-    const float *urow = Us + j * OB + lane;
-    float u[4];
+  const float4 *u4 = reinterpret_cast<const float4 *>(Up + J * QUROW + p * QUP);
+  const float iu = inv[J];
+  const float wj = __shfl_sync(0xffffffffu, S.w[io], quad | po);
+  // w/scale as a product with the group's reciprocal: it can differ from
+  // the quotient only within an ulp of a rounding tie
+  const float q = fminf(fmaxf(rintf(wj * S.rscale) + S.zero, 0.f), maxq);
+  const float wh = S.scale * (q - S.zero);
+  const float e = (wj - wh) * iu;
+  {
+    const uint32_t qi = static_cast<uint32_t>(q);
+    constexpr int bit = J * BITS, k = bit / 32, s = bit % 32;
+    S.cw[k] |= qi << s;
+    if constexpr (s + BITS > 32) S.cw[k + 1] |= qi >> (32 - s);
+  }
 #pragma unroll
-    for (int s = SLOT; s < 4; ++s) u[s] = urow[32 * s];
-    const float iu = inv[j];
+  for (int a = io / 4; a < QNI / 4; ++a) {
+    const float4 u = u4[a];
+    const float uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float wj = __shfl_sync(0xffffffffu, w[r][SLOT], jj);
-      // w/scale as a product with the group's reciprocal: it can differ from
-      // the quotient only within an ulp of a rounding tie
-      const float q = fminf(fmaxf(rintf(wj * rscale[r]) + zero[r], 0.f), maxq);
-      const float wh = scale[r] * (q - zero[r]);
-      const float e = (wj - wh) * iu;
-      if (lane > jj) w[r][SLOT] = fmaf(-e, u[SLOT], w[r][SLOT]);
-#pragma unroll
-      for (int s = SLOT + 1; s < 4; ++s) w[r][s] = fmaf(-e, u[s], w[r][s]);
-      if (lane == jj) {
-        w[r][SLOT] = wh;
-        err[r][SLOT] = e;
-        qs[r][j] = static_cast<uint8_t>(q);
+    for (int c = 0; c < 4; ++c) {
+      const int i = 4 * a + c;
+      if (i == io) {
+        // the column itself: the owner keeps w_hat and the error, the lanes
+        // right of it in the quad update their column of the same i
+        if (p > po) S.w[i] = fmaf(-e, uu[c], S.w[i]);
+        else if (p == po) {
+          S.w[i] = wh;
+          S.err[i] = e;
+        }
+      } else if (i > io) {
+        S.w[i] = fmaf(-e, uu[c], S.w[i]);
       }
     }
   }
 }
 
-// One 128-column block for OROWS rows per CTA. Each warp sweeps its 4 rows
-// together (independent dependency chains), lane l holding columns
-// l, l+32, l+64, l+96 of each row.
+template <int BITS, int... J>
+__device__ __forceinline__ void obs_sweep(std::integer_sequence<int, J...>,
+                                          SweepState<BITS> &S, const float *Up,
+                                          const float *inv, int p, int quad, int group,
+                                          const GroupOut &go) {
+  (obs_column<BITS, J>(S, Up, inv, p, quad, group, go), ...);
+}
+
+// One 128-column block for OROWS rows per CTA (8 rows per warp).
+template <int BITS>
 __global__ void __launch_bounds__(OTHREADS)
     obs_block_kernel(float *__restrict__ W, int64_t ldw,
                      const float *__restrict__ U, int64_t ldu, int64_t j0,
-                     int64_t d_out, int bits, int group,
+                     int64_t d_out, int group,
                      float *__restrict__ E, int64_t lde, int64_t e_col,
                      uint32_t *__restrict__ codes, int64_t ldq,
                      float *__restrict__ scales, uint8_t *__restrict__ zeros,
                      int64_t ngroups) {
-  extern __shared__ float Us[];                 // OB x OB, then 1/U[j][j]
-  float *inv = Us + OB * OB;
-  __shared__ uint8_t qsm[OTHREADS / 32][RPW][OB];
+  extern __shared__ __align__(16) float Up[];  // Up[j][p][i] = U[j][4i + p]
+  float *inv = Up + OB * QUROW;                // 1/U[j][j]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = lane & (QLPR - 1), quad = lane & ~(QLPR - 1);
+  const int64_t row = int64_t(blockIdx.x) * OROWS + warp * (32 / QLPR) + lane / QLPR;
+  const bool ok = row < d_out;
   for (int e = threadIdx.x; e < OB * OB; e += OTHREADS) {
     const int r = e / OB, c = e % OB;
-    Us[e] = U[(j0 + r) * ldu + j0 + c];
+    Up[r * QUROW + (c % QLPR) * QUP + c / QLPR] = U[(j0 + r) * ldu + j0 + c];
+  }
+  SweepState<BITS> S;
+#pragma unroll
+  for (int i = 0; i < QNI; ++i) {
+    S.w[i] = ok ? W[row * ldw + j0 + QLPR * i + p] : 0.f;
+    S.err[i] = 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < SweepState<BITS>::NW; ++k) S.cw[k] = 0u;
+  S.scale = 1.f;
+  S.rscale = 1.f;
+  S.zero = 0.f;
+  __syncthreads();
+  if (threadIdx.x < OB) {
+    const int j = threadIdx.x;
+    inv[j] = 1.f / Up[j * QUROW + (j % QLPR) * QUP + j / QLPR];
   }
   __syncthreads();
-  if (threadIdx.x < OB) inv[threadIdx.x] = 1.f / Us[threadIdx.x * OB + threadIdx.x];
-  __syncthreads();
-  const float maxq = static_cast<float>((1 << bits) - 1);
-  const int64_t row0 = int64_t(blockIdx.x) * OROWS + warp * RPW;
-  float w[RPW][4], err[RPW][4];
+  const GroupOut go{scales + row * ngroups, zeros + row * ngroups, j0 / group,
+                    p == 0 && ok};
+  obs_sweep<BITS>(std::make_integer_sequence<int, OB>{}, S, Up, inv, p, quad, group, go);
+  if (!ok) return;
 #pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-    const bool ok = row0 + r < d_out;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      w[r][s] = ok ? W[(row0 + r) * ldw + j0 + lane + 32 * s] : 0.f;
-      err[r][s] = 0.f;
-    }
+  for (int i = 0; i < QNI; ++i) {
+    W[row * ldw + j0 + QLPR * i + p] = S.w[i];
+    E[row * lde + e_col + QLPR * i + p] = S.err[i];
   }
-  float scale[RPW], rscale[RPW], zero[RPW];
-  uint8_t (*qs)[OB] = qsm[warp];
-  obs_chunk<0>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
-               d_out, j0, scales, zeros, ngroups);
-  obs_chunk<1>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
-               d_out, j0, scales, zeros, ngroups);
-  obs_chunk<2>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
-               d_out, j0, scales, zeros, ngroups);
-  obs_chunk<3>(w, err, scale, rscale, zero, Us, inv, qs, lane, group, maxq, row0,
-               d_out, j0, scales, zeros, ngroups);
-  __syncwarp();
-  const int nwords = OB * bits / 32;
+  uint32_t *cr = codes + row * ldq + (j0 * BITS) / 32;
 #pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-    const int64_t row = row0 + r;
-    if (row >= d_out) break;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      W[row * ldw + j0 + lane + 32 * s] = w[r][s];
-      E[row * lde + e_col + lane + 32 * s] = err[r][s];
-    }
-    if (lane < nwords) {
-      uint32_t word = 0;
-      const int bit0 = 32 * lane;
-      const int c_lo = bit0 / bits, c_hi = min(OB - 1, (bit0 + 31) / bits);
-      for (int c = c_lo; c <= c_hi; ++c) {
-        const int sh = c * bits - bit0;
-        const uint32_t code = qsm[warp][r][c];
-        word |= sh >= 0 ? (code << sh) : (code >> (-sh));
-      }
-      codes[row * ldq + (j0 * bits) / 32 + lane] = word;
-    }
-  }
+  for (int k = 0; k < SweepState<BITS>::NW; ++k)
+    if (k / BITS == p) cr[k] = S.cw[k];
 }
 
 __global__ void diff_inplace_kernel(float *__restrict__ A, int64_t lda,
@@ -207,20 +222,27 @@ kronq_status quantize_view(cudaStream_t st, const kronq_opts &o, const QuantView
   const size_t scr_bytes = ws_bytes - e_bytes;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(obs_block_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             OSMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(obs_block_kernel<2>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, OSMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(obs_block_kernel<3>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, OSMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(obs_block_kernel<4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, OSMEM) != cudaSuccess)
       return KRONQ_ERR_CUDA;
     attr_done = true;
   }
+  auto block_kernel = o.bits == 2 ? obs_block_kernel<2>
+                      : o.bits == 3 ? obs_block_kernel<3>
+                                    : obs_block_kernel<4>;
+  if (o.bits < 2 || o.bits > 4) return KRONQ_ERR_INVALID_ARG;
   float *W = v.W;
   const float *U = v.U;
   const unsigned grid = static_cast<unsigned>(ceil_div(d_out, OROWS));
   for (int64_t sb0 = 0; sb0 < n; sb0 += S) {
     const int64_t sb1 = kq_min<int64_t>(n, sb0 + S);
     for (int64_t j0 = sb0; j0 < sb1; j0 += OB) {
-      obs_block_kernel<<<grid, OTHREADS, OSMEM, st>>>(
-          W, v.ldw, U, v.ldu, j0, d_out, o.bits, o.group, E, S, j0 - sb0, v.codes,
+      block_kernel<<<grid, OTHREADS, OSMEM, st>>>(
+          W, v.ldw, U, v.ldu, j0, d_out, o.group, E, S, j0 - sb0, v.codes,
           v.ldq, v.scales, v.zeros, v.lds);
       KQ_CHECK_LAUNCH();
       if (j0 + OB < sb1) {
