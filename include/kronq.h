@@ -351,6 +351,11 @@ const char *kronq_status_string(kronq_status s);
  * thread-safe, never fails. */
 uint64_t kronq_kernel_launches(void);
 
+/* Diagnostics: the CUDA runtime's description of the last CUDA call that made
+ * an entry point return KRONQ_ERR_CUDA in this process ("no error" if none).
+ * Static string owned by the CUDA runtime; host call, never fails. */
+const char *kronq_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -281,4 +281,8 @@ kronq_status kronq_allocate_bits(const double *score, const int64_t *numel,
 
 uint64_t kronq_kernel_launches(void) { return launches(); }
 
+const char *kronq_last_cuda_error(void) {
+  return cudaGetErrorString(static_cast<cudaError_t>(last_cuda_error()));
+}
+
 }  // extern "C"

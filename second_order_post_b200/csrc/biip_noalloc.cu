@@ -34,7 +34,7 @@ std::mutex g_scratch_mu;
 // Device address of g_biip_scratch on the current device (set up once).
 kronq_status scratch_on_current_device(void **out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KRONQ_ERR_CUDA;
+  KQ_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return KRONQ_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_addr[dev] == nullptr) {

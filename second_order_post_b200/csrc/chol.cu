@@ -60,25 +60,33 @@ __global__ void damping_kernel(const float *H, int64_t d, float damp_rel,
 // the left factor right of it. U = D^-1/2 X.
 //
 // Each thread keeps one 4x4 tile of the upper triangle in registers. Pivots
-// are taken four at a time (the pivot block J = [j0, j0+4) is one tile): the
-// owners of tile column J publish their tiles (M[i][J], i < j0+4, the pivot
-// block included) and the owners of tile row J theirs (M[J][k], k >= j0+4),
-// and after one barrier every thread replays the four pivots on its own tile.
-// Within the block, pivot jj changes the published values that later pivots
-// of the block read; each thread carries those along itself:
-//     M[i][j'] -= (M[i][jj] / p) M[j'][jj]      (its rows, j' < jj in J)
-//     b_j'[k]  -= (M[j'][jj] / p) b_jj[k]        (its columns outside J)
-// and factors the 4x4 pivot block redundantly, so a block costs one barrier.
+// are taken four at a time (the pivot block J = [j0, j0+4) is one tile), in
+// two phases separated by barriers:
+//   A. The owners of tile column J and tile row J have published them. Every
+//      phase-A thread factors the 4x4 pivot block (redundantly, in registers),
+//      then thread i < j0 replays the four pivots on row i of the column
+//      panel and thread k >= j0+4 on column k of the row panel. Row i gives
+//      l_q[i] and the value b_q[i] = M[i][j0+q] that pivot q reads in column
+//      i; column k gives b_q[k] = M[j0+q][k], final once pivot q is reached.
+//   B. Every other tile above the block row takes the four pivots as one
+//      rank-4 update, M[i][k] -= sum_q l_q[i] b_q[k] (q = 3 .. 0, the order of
+//      the one-pivot sweep); the panel owners take their final values back.
+// Each phase-A chain is one row or column, so a block costs two barriers and
+// no thread replays more than its own panel entry.
 constexpr int TT = 4;                          // tile edge owned by a thread
 constexpr int NT = NB / TT;                    // tile rows and columns
 constexpr int NTILES = NT * (NT + 1) / 2;      // upper tiles (I <= K)
 constexpr int LTHREADS = (NTILES + 31) / 32 * 32;
+static_assert(LTHREADS >= 2 * NB, "phase A needs a thread per panel row and column");
 
 __global__ void __launch_bounds__(LTHREADS)
     chol_leaf_kernel(float *__restrict__ H, int64_t ld, int64_t off,
                      const float *__restrict__ lambda, int32_t *info) {
-  __shared__ __align__(16) float colbuf[2][NB][TT];  // M[i][J], row i
+  __shared__ __align__(16) float colbuf[2][NB][TT];  // M[i][J], rows i < j0+4
   __shared__ __align__(16) float rowbuf[2][TT][NB];  // M[J][k]
+  __shared__ __align__(16) float Ls[NB][TT];         // l_q[i], rows i < j0
+  __shared__ __align__(16) float Bs[TT][NB];         // b_q[k], k outside J
+  __shared__ __align__(16) float blkf[TT][TT];       // the pivot block, factored
   __shared__ float piv[NB];
   const int t = threadIdx.x;
   const bool own = t < NTILES;
@@ -127,34 +135,20 @@ __global__ void __launch_bounds__(LTHREADS)
   __syncthreads();
   bool bad = false;
   for (int Tj = NT - 1; Tj >= 0; --Tj) {
-    const int j0 = TT * Tj, bs_ = Tj & 1;
-    if (own && I <= Tj) {
-      float blk[TT][TT], ar[TT][TT], bsrc[TT][TT];
+    const int j0 = TT * Tj, par = Tj & 1;
+    // ---------------- phase A
+    if (t < 2 * NB) {
+      float blk[TT][TT];
 #pragma unroll
       for (int a = 0; a < TT; ++a) {
-        const float4 v = *reinterpret_cast<const float4 *>(&colbuf[bs_][j0 + a][0]);
+        const float4 v = *reinterpret_cast<const float4 *>(&colbuf[par][j0 + a][0]);
         blk[a][0] = v.x; blk[a][1] = v.y; blk[a][2] = v.z; blk[a][3] = v.w;
-        const float4 w = *reinterpret_cast<const float4 *>(&colbuf[bs_][r0 + a][0]);
-        ar[a][0] = w.x; ar[a][1] = w.y; ar[a][2] = w.z; ar[a][3] = w.w;
       }
-      const bool in_blk = K == Tj;
-      if (K < Tj) {  // columns left of J: b_jj[k] = M[k][jj]
-#pragma unroll
-        for (int kk = 0; kk < TT; ++kk) {
-          const float4 v = *reinterpret_cast<const float4 *>(&colbuf[bs_][c0 + kk][0]);
-          bsrc[0][kk] = v.x; bsrc[1][kk] = v.y; bsrc[2][kk] = v.z; bsrc[3][kk] = v.w;
-        }
-      } else if (K > Tj) {  // columns right of J: b_jj[k] = M[jj][k]
-#pragma unroll
-        for (int q = 0; q < TT; ++q) {
-          const float4 v = *reinterpret_cast<const float4 *>(&rowbuf[bs_][q][c0]);
-          bsrc[q][0] = v.x; bsrc[q][1] = v.y; bsrc[q][2] = v.z; bsrc[q][3] = v.w;
-        }
-      }
+      float rp[TT], bq[TT][TT], lq[TT][TT];
 #pragma unroll
       for (int q = TT - 1; q >= 0; --q) {
         const float p = blk[q][q];
-        const float rp = __frcp_rn(p);
+        rp[q] = __frcp_rn(p);
         if (t == 0) {
           piv[j0 + q] = p;
           if (!(p > 0.f) || !isfinite(p)) {
@@ -163,46 +157,98 @@ __global__ void __launch_bounds__(LTHREADS)
             bad = true;
           }
         }
-        float l[TT], b[TT];
-#pragma unroll
-        for (int ii = 0; ii < TT; ++ii) l[ii] = r0 + ii < j0 + q ? ar[ii][q] * rp : 0.f;
-#pragma unroll
-        for (int kk = 0; kk < TT; ++kk)
-          b[kk] = in_blk ? (kk < q ? blk[kk][q] : kk == q ? p + 1.f : blk[q][kk])
-                         : bsrc[q][kk];
-#pragma unroll
-        for (int ii = 0; ii < TT; ++ii)
-#pragma unroll
-          for (int kk = 0; kk < TT; ++kk) m[ii][kk] = fmaf(-l[ii], b[kk], m[ii][kk]);
-        // carry the pivot into the values that the later pivots q' < q read
-#pragma unroll
-        for (int qq = 0; qq < q; ++qq) {
-          const float c = blk[qq][q] * rp;
-#pragma unroll
-          for (int ii = 0; ii < TT; ++ii) ar[ii][qq] = fmaf(-ar[ii][q] * rp, blk[qq][q], ar[ii][qq]);
-          if (!in_blk) {
-#pragma unroll
-            for (int kk = 0; kk < TT; ++kk) bsrc[qq][kk] = fmaf(-c, bsrc[q][kk], bsrc[qq][kk]);
-          }
-        }
         float colq[TT], rowq[TT];
 #pragma unroll
         for (int a = 0; a < TT; ++a) {
           colq[a] = blk[a][q];
           rowq[a] = blk[q][a];
+          bq[q][a] = a < q ? colq[a] : a == q ? p + 1.f : rowq[a];
+          lq[q][a] = a < q ? colq[a] * rp[q] : 0.f;
         }
 #pragma unroll
         for (int a = 0; a < q; ++a) {
-          const float la = colq[a] * rp;
+          const float la = lq[q][a];
 #pragma unroll
-          for (int bb = a; bb < TT; ++bb) {
-            const float v = bb < q ? colq[bb] : bb == q ? p + 1.f : rowq[bb];
-            blk[a][bb] = fmaf(-la, v, blk[a][bb]);
+          for (int bb = a; bb < TT; ++bb) blk[a][bb] = fmaf(-la, bq[q][bb], blk[a][bb]);
+        }
+      }
+      if (t < NB) {
+        const int i = t;
+        if (i < j0) {
+          const float4 v = *reinterpret_cast<const float4 *>(&colbuf[par][i][0]);
+          float P[TT] = {v.x, v.y, v.z, v.w};
+          float Lr[TT];
+#pragma unroll
+          for (int q = TT - 1; q >= 0; --q) {
+            const float l = P[q] * rp[q];
+            Lr[q] = l;
+            Bs[q][i] = P[q];
+#pragma unroll
+            for (int a = 0; a < TT; ++a) P[a] = fmaf(-l, bq[q][a], P[a]);
           }
+          *reinterpret_cast<float4 *>(&Ls[i][0]) = make_float4(Lr[0], Lr[1], Lr[2], Lr[3]);
+          *reinterpret_cast<float4 *>(&colbuf[par][i][0]) = make_float4(P[0], P[1], P[2], P[3]);
+        } else if (i == j0) {
+          // (not into colbuf: the other phase-A threads may still read it)
+#pragma unroll
+          for (int a = 0; a < TT; ++a)
+            *reinterpret_cast<float4 *>(&blkf[a][0]) =
+                make_float4(blk[a][0], blk[a][1], blk[a][2], blk[a][3]);
+        }
+      } else {
+        const int k = t - NB;
+        if (k >= j0 + TT) {
+          float R[TT];
+#pragma unroll
+          for (int a = 0; a < TT; ++a) R[a] = rowbuf[par][a][k];
+#pragma unroll
+          for (int q = TT - 1; q >= 0; --q) {
+            Bs[q][k] = R[q];
+#pragma unroll
+            for (int a = 0; a < q; ++a) R[a] = fmaf(-lq[q][a], R[q], R[a]);
+          }
+#pragma unroll
+          for (int a = 0; a < TT; ++a) rowbuf[par][a][k] = R[a];
         }
       }
     }
-    if (own && Tj > 0) publish(Tj - 1);
+    __syncthreads();
+    // ---------------- phase B, then the panels of the next block
+    if (own) {
+      if (I < Tj && K != Tj) {
+        float l[TT][TT], b[TT][TT];  // l[ii][q], b[q][kk]
+#pragma unroll
+        for (int ii = 0; ii < TT; ++ii) {
+          const float4 v = *reinterpret_cast<const float4 *>(&Ls[r0 + ii][0]);
+          l[ii][0] = v.x; l[ii][1] = v.y; l[ii][2] = v.z; l[ii][3] = v.w;
+        }
+#pragma unroll
+        for (int q = 0; q < TT; ++q) {
+          const float4 v = *reinterpret_cast<const float4 *>(&Bs[q][c0]);
+          b[q][0] = v.x; b[q][1] = v.y; b[q][2] = v.z; b[q][3] = v.w;
+        }
+#pragma unroll
+        for (int q = TT - 1; q >= 0; --q)
+#pragma unroll
+          for (int ii = 0; ii < TT; ++ii)
+#pragma unroll
+            for (int kk = 0; kk < TT; ++kk) m[ii][kk] = fmaf(-l[ii][q], b[q][kk], m[ii][kk]);
+      } else if (K == Tj) {
+#pragma unroll
+        for (int ii = 0; ii < TT; ++ii) {
+          const float4 v = I == Tj ? *reinterpret_cast<const float4 *>(&blkf[ii][0])
+                                   : *reinterpret_cast<const float4 *>(&colbuf[par][r0 + ii][0]);
+          m[ii][0] = v.x; m[ii][1] = v.y; m[ii][2] = v.z; m[ii][3] = v.w;
+        }
+      } else if (I == Tj) {
+#pragma unroll
+        for (int ii = 0; ii < TT; ++ii) {
+          const float4 v = *reinterpret_cast<const float4 *>(&rowbuf[par][ii][c0]);
+          m[ii][0] = v.x; m[ii][1] = v.y; m[ii][2] = v.z; m[ii][3] = v.w;
+        }
+      }
+      if (Tj > 0) publish(Tj - 1);
+    }
     __syncthreads();
   }
   if (own) {
@@ -262,9 +308,8 @@ kronq_status chol_streams(CholStreams **out) {
   CholStreams &cs = per_dev[dev];
   if (!cs.ready) {
     int lo = 0, hi = 0;
-    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return KRONQ_ERR_CUDA;
-    if (cudaStreamCreateWithPriority(&cs.main, cudaStreamNonBlocking, hi) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
+    KQ_CUDA(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+    KQ_CUDA(cudaStreamCreateWithPriority(&cs.main, cudaStreamNonBlocking, hi));
     if (cudaEventCreateWithFlags(&cs.fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&cs.join_main, cudaEventDisableTiming) != cudaSuccess)
       return KRONQ_ERR_CUDA;
@@ -324,8 +369,7 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
     g.kflags = KR_B_LOWER;
     KQ_TRY(gemm_f32(c.side[depth], g, c.scr_side[depth], c.scr_side_bytes[depth], c.info));
   }
-  if (cudaEventRecord(c.ev_t[depth], c.side[depth]) != cudaSuccess)
-    return KRONQ_ERR_CUDA;
+  KQ_CUDA(cudaEventRecord(c.ev_t[depth], c.side[depth]));
   }
   {
     GemmArgs g;  // A11 -= V Vᵀ (tiles on or above the diagonal)
@@ -340,12 +384,11 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
   KQ_TRY(rinv(c, off, h, depth + 1));  // A11 -> U11
   if (keep_r) {
     // the caller's OBS crosses the halves with R12 = V itself
-    if (cudaMemcpy2DAsync(B12, static_cast<size_t>(d) * 4, V, static_cast<size_t>(m) * 4,
+    KQ_CUDA(cudaMemcpy2DAsync(B12, static_cast<size_t>(d) * 4, V, static_cast<size_t>(m) * 4,
                           static_cast<size_t>(m) * 4, static_cast<size_t>(h),
-                          cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
+                          cudaMemcpyDeviceToDevice, c.st));
   } else {
-  if (cudaStreamWaitEvent(c.st, c.ev_t[depth], 0) != cudaSuccess) return KRONQ_ERR_CUDA;
+  KQ_CUDA(cudaStreamWaitEvent(c.st, c.ev_t[depth], 0));
   {
     GemmArgs g;  // U12 = -U11 T : U11[i][k] == 0 for k < i
     g.M = h; g.N = m; g.K = h;
@@ -359,10 +402,9 @@ kronq_status rinv(const Ctx &c, int64_t off, int64_t n, int depth) {
   }
   // zeros below the diagonal of this node (the leaves zero their own blocks):
   // triangular operands of the parents' products read U as 128 x 256 tiles
-  if (cudaMemset2DAsync(c.H + (off + h) * d + off, static_cast<size_t>(d) * 4, 0,
+  KQ_CUDA(cudaMemset2DAsync(c.H + (off + h) * d + off, static_cast<size_t>(d) * 4, 0,
                         static_cast<size_t>(h) * 4, static_cast<size_t>(m),
-                        c.st) != cudaSuccess)
-    return KRONQ_ERR_CUDA;
+                        c.st));
   return KRONQ_OK;
 }
 
@@ -442,7 +484,7 @@ kronq_status chol_run(cudaStream_t st, float *H, int64_t d, float damp_rel,
       cudaStreamWaitEvent(cs->main, cs->fork, 0) != cudaSuccess)
     return KRONQ_ERR_CUDA;
   for (int k = 0; k < depths; ++k)
-    if (cudaStreamWaitEvent(cs->side[k], cs->fork, 0) != cudaSuccess) return KRONQ_ERR_CUDA;
+    KQ_CUDA(cudaStreamWaitEvent(cs->side[k], cs->fork, 0));
   damping_kernel<<<1, 1024, 0, c.st>>>(H, d, damp_rel, lambda, info);
   KQ_CHECK_LAUNCH();
   KQ_TRY(rinv(c, 0, d, 0));

@@ -20,11 +20,21 @@ __host__ __device__ __forceinline__ T kq_max(T a, T b) { return a < b ? b : a; }
 // Counts every kernel the library launches (reported by kronq_kernel_launches).
 void count_launch();
 
+// Records a failed CUDA call (reported by kronq_last_cuda_error) and returns
+// KRONQ_ERR_CUDA.
+kronq_status cuda_fail(cudaError_t e);
+
 #define KQ_CHECK_LAUNCH()                                                      \
   do {                                                                         \
     count_launch();                                                            \
     cudaError_t e_ = cudaGetLastError();                                       \
-    if (e_ != cudaSuccess) return KRONQ_ERR_CUDA;                              \
+    if (e_ != cudaSuccess) return ::kronq::cuda_fail(e_);                      \
+  } while (0)
+
+#define KQ_CUDA(expr)                                                          \
+  do {                                                                         \
+    cudaError_t e_ = (expr);                                                   \
+    if (e_ != cudaSuccess) return ::kronq::cuda_fail(e_);                      \
   } while (0)
 
 #define KQ_TRY(expr)                                                           \

@@ -330,10 +330,9 @@ kronq_status cov_bf16(cudaStream_t st, const __nv_bfloat16 *A, int64_t n,
   const int64_t tiles = nt * (nt + 1) / 2;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(cov_bf16_kernel,
+    KQ_CUDA(cudaFuncSetAttribute(cov_bf16_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CSMEM) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
+                             CSMEM));
     attr_done = true;
   }
   cov_bf16_kernel<<<static_cast<unsigned>(tiles), CTHREADS, CSMEM, st>>>(

@@ -430,9 +430,8 @@ kronq_status launch(cudaStream_t st, const GemmArgs &g, int32_t *info,
   if (tiles > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
+    KQ_CUDA(cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM));
     attr_done = true;
   }
   GemmP p;
@@ -592,8 +591,7 @@ kronq_status split_operand(cudaStream_t st, const float *X, int64_t ld, bool mn,
         X, ld, rows, K, hi, lo, ldp, inv, vec);
     KQ_CHECK_LAUNCH();
   } else {
-    if (cudaMemsetAsync(maxbits, 0, static_cast<size_t>(rows) * 4, st) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
+    KQ_CUDA(cudaMemsetAsync(maxbits, 0, static_cast<size_t>(rows) * 4, st));
     const int64_t kchunk = 256;
     dim3 gm(static_cast<unsigned>(ceil_div(rows, 256)),
             static_cast<unsigned>(ceil_div(K, kchunk)));

@@ -55,6 +55,7 @@ kronq_status launch_sensitivity(cudaStream_t st, const float *hx, int64_t dx,
                                 const float *hg, int64_t dg, double *out);
 kronq_status launch_set_int(cudaStream_t st, int32_t *p, int32_t v);
 uint64_t launches();
+int last_cuda_error();
 
 // ---------------------------------------------------------------- Cholesky
 size_t chol_ws_bytes(int64_t d);

@@ -64,7 +64,7 @@ kronq_status layer_loss(cudaStream_t st, const float *W_ref, const float *W_hat,
   h.B = D; h.ldb = d_in; h.b_mn = true;
   h.C = Q; h.ldc = d_in;
   KQ_TRY(gemm_f32(st, h, scr, scr_bytes, nullptr));
-  if (cudaMemsetAsync(loss, 0, sizeof(double), st) != cudaSuccess) return KRONQ_ERR_CUDA;
+  KQ_CUDA(cudaMemsetAsync(loss, 0, sizeof(double), st));
   dot_kernel<<<blocks, 256, 0, st>>>(P, Q, n, loss);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;

@@ -58,11 +58,20 @@ std::atomic<uint64_t> g_launches{0};
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+namespace {
+std::atomic<int> g_last_cuda{0};
+}
+kronq_status cuda_fail(cudaError_t e) {
+  g_last_cuda.store(static_cast<int>(e), std::memory_order_relaxed);
+  return KRONQ_ERR_CUDA;
+}
+int last_cuda_error() { return g_last_cuda.load(std::memory_order_relaxed); }
+
 uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
 kronq_status require_sm100() {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KRONQ_ERR_CUDA;
+  KQ_CUDA(cudaGetDevice(&dev));
   static int checked_dev = -1;
   static bool ok = false;
   if (checked_dev != dev) {

@@ -60,6 +60,8 @@ def make_opts(bits=4, group=128, block=128, damp_rel=0.01, scale_exp=0.25,
 class KronqError(RuntimeError):
     def __init__(self, fn, status):
         msg = _lib.kronq_status_string(status).decode()
+        if status == KRONQ_ERR_CUDA:
+            msg += ": " + _lib.kronq_last_cuda_error().decode()
         super().__init__(f"{fn}: {msg} (status {status})")
         self.status = status
 
@@ -88,6 +90,7 @@ _SIGS = {
     "kronq_allocate_bits": [_p, _p, ctypes.c_int, _d, _p],
     "kronq_status_string": [ctypes.c_int],
     "kronq_kernel_launches": [],
+    "kronq_last_cuda_error": [],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -98,6 +101,7 @@ _lib.kronq_gemm_f32_workspace_bytes.restype = ctypes.c_size_t
 _lib.kronq_chol_split_point.restype = ctypes.c_int64
 _lib.kronq_status_string.restype = ctypes.c_char_p
 _lib.kronq_kernel_launches.restype = ctypes.c_uint64
+_lib.kronq_last_cuda_error.restype = ctypes.c_char_p
 
 
 def _check(fn, st):

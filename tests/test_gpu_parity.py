@@ -102,6 +102,8 @@ BIIP_CASES = [
     # d_out, d_in, rot_out, rot_in, flags, w dtype
     (256, 256, (256, 1), (256, 1), 0, torch.float32),
     (256, 896, (256, 1), (32, 28), 0, torch.float32),
+    # 1792 rows of H_X over 148 persistent CTAs: uneven unit counts per CTA
+    (1024, 1792, (1024, 1), (64, 28), 0, torch.float32),
     (688, 256, (4, 172), (256, 1), 0, torch.bfloat16),
     (344, 1376, (2, 172), (8, 172), 0, torch.float32),
     (128, 4096, (128, 1), (4096, 1), 0, torch.bfloat16),
