@@ -3,15 +3,15 @@
 // and H_G does not enter it, so rows are independent given U; wmrh §五:
 // W2/W3/W4 with 128-column groups].
 //
-// Per 128-column block j0 (one launch of obs_block_kernel): four lanes share
-// one row, lane p of the quad holding the columns 4i + p (i < 32) in
+// Per 128-column block j0 (one launch of obs_block_kernel): eight lanes share
+// one row, lane p of the group holding the columns 8i + p (i < 16) in
 // registers, so that every lane has about the same number of updates left at
 // any column. U[j0:j0+128, j0:j0+128] sits in shared memory, permuted so that
 // each lane's columns of a U row are contiguous. The sweep over the block's
 // 128 columns is unrolled, so every register index is a compile-time
 // constant. For each column j: group (scale, zero) at a group start,
-// q = clamp(rint(w/scale)+zero), err = (w - w_hat)/U[j][j] (all four lanes
-// of the quad compute them from the owner's weight), w_k -= err * U[j][k] for
+// q = clamp(rint(w/scale)+zero), err = (w - w_hat)/U[j][j] (all lanes of
+// the row's group compute them from the owner's weight), w_k -= err * U[j][k] for
 // the block's k > j. The errors go to E; the columns right of the block are
 // updated lazily by 3xTF32 GEMMs: within a super-block of S columns after
 // every block (W[:, blk_end:sb_end] -= E_blk U[blk, blk_end:sb_end]), and
@@ -26,9 +26,9 @@ namespace kronq {
 namespace {
 
 constexpr int OB = 128;                    // block width
-constexpr int QLPR = 4;                    // lanes per row
+constexpr int QLPR = 8;                    // lanes per row
 constexpr int QNI = OB / QLPR;             // columns (registers) per lane
-constexpr int QWARPS = 4;
+constexpr int QWARPS = 8;
 constexpr int OTHREADS = 32 * QWARPS;
 constexpr int OROWS = QWARPS * (32 / QLPR);  // rows per CTA
 constexpr int QUP = QNI + 4;               // one lane's run of a U row (padded)
@@ -57,7 +57,7 @@ struct GroupOut {
 // Column J of the block (every register index is a compile-time constant).
 template <int BITS, int J>
 __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
-                                           const float *inv, int p, int quad,
+                                           const float *inv, int p, int grp,
                                            int group, const GroupOut &go) {
   constexpr int io = J / QLPR, po = J % QLPR;
   constexpr float maxq = static_cast<float>((1 << BITS) - 1);
@@ -95,7 +95,7 @@ __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
   }
   const float4 *u4 = reinterpret_cast<const float4 *>(Up + J * QUROW + p * QUP);
   const float iu = inv[J];
-  const float wj = __shfl_sync(0xffffffffu, S.w[io], quad | po);
+  const float wj = __shfl_sync(0xffffffffu, S.w[io], grp | po);
   // w/scale as a product with the group's reciprocal: it can differ from
   // the quotient only within an ulp of a rounding tie
   const float q = fminf(fmaxf(rintf(wj * S.rscale) + S.zero, 0.f), maxq);
@@ -116,7 +116,7 @@ __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
       const int i = 4 * a + c;
       if (i == io) {
         // the column itself: the owner keeps w_hat and the error, the lanes
-        // right of it in the quad update their column of the same i
+        // right of it in the row's group update their column of the same i
         if (p > po) S.w[i] = fmaf(-e, uu[c], S.w[i]);
         else if (p == po) {
           S.w[i] = wh;
@@ -132,12 +132,12 @@ __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
 template <int BITS, int... J>
 __device__ __forceinline__ void obs_sweep(std::integer_sequence<int, J...>,
                                           SweepState<BITS> &S, const float *Up,
-                                          const float *inv, int p, int quad, int group,
+                                          const float *inv, int p, int grp, int group,
                                           const GroupOut &go) {
-  (obs_column<BITS, J>(S, Up, inv, p, quad, group, go), ...);
+  (obs_column<BITS, J>(S, Up, inv, p, grp, group, go), ...);
 }
 
-// One 128-column block for OROWS rows per CTA (8 rows per warp).
+// One 128-column block for OROWS rows per CTA (32 / QLPR rows per warp).
 template <int BITS>
 __global__ void __launch_bounds__(OTHREADS)
     obs_block_kernel(float *__restrict__ W, int64_t ldw,
@@ -147,21 +147,40 @@ __global__ void __launch_bounds__(OTHREADS)
                      uint32_t *__restrict__ codes, int64_t ldq,
                      float *__restrict__ scales, uint8_t *__restrict__ zeros,
                      int64_t ngroups) {
-  extern __shared__ __align__(16) float Up[];  // Up[j][p][i] = U[j][4i + p]
+  extern __shared__ __align__(16) float Up[];  // Up[j][p][i] = U[j][QLPR*i + p]
   float *inv = Up + OB * QUROW;                // 1/U[j][j]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = lane & (QLPR - 1), quad = lane & ~(QLPR - 1);
+  const int p = lane & (QLPR - 1), grp = lane & ~(QLPR - 1);
   const int64_t row = int64_t(blockIdx.x) * OROWS + warp * (32 / QLPR) + lane / QLPR;
   const bool ok = row < d_out;
-  for (int e = threadIdx.x; e < OB * OB; e += OTHREADS) {
-    const int r = e / OB, c = e % OB;
-    Up[r * QUROW + (c % QLPR) * QUP + c / QLPR] = U[(j0 + r) * ldu + j0 + c];
-  }
   SweepState<BITS> S;
 #pragma unroll
   for (int i = 0; i < QNI; ++i) {
     S.w[i] = ok ? W[row * ldw + j0 + QLPR * i + p] : 0.f;
     S.err[i] = 0.f;
+  }
+  // U block: float4 loads of a row's 4 consecutive columns (one per lane
+  // phase), eight in flight per thread, scattered into the permuted layout
+  constexpr int C4 = OB / 4;                        // float4s per U row
+  constexpr int BATCH = 8;
+  static_assert((OB * C4) % (OTHREADS * BATCH) == 0, "U block batches");
+  for (int e0 = threadIdx.x; e0 < OB * C4; e0 += OTHREADS * BATCH) {
+    float4 v[BATCH];
+#pragma unroll
+    for (int b = 0; b < BATCH; ++b) {
+      const int e = e0 + b * OTHREADS, r = e / C4, c4 = e % C4;
+      v[b] = __ldg(reinterpret_cast<const float4 *>(U + (j0 + r) * ldu + j0) + c4);
+    }
+#pragma unroll
+    for (int b = 0; b < BATCH; ++b) {
+      const int e = e0 + b * OTHREADS, r = e / C4, c4 = e % C4;
+      const float vv[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = 4 * c4 + q;
+        Up[r * QUROW + (c % QLPR) * QUP + c / QLPR] = vv[q];
+      }
+    }
   }
 #pragma unroll
   for (int k = 0; k < SweepState<BITS>::NW; ++k) S.cw[k] = 0u;
@@ -176,7 +195,7 @@ __global__ void __launch_bounds__(OTHREADS)
   __syncthreads();
   const GroupOut go{scales + row * ngroups, zeros + row * ngroups, j0 / group,
                     p == 0 && ok};
-  obs_sweep<BITS>(std::make_integer_sequence<int, OB>{}, S, Up, inv, p, quad, group, go);
+  obs_sweep<BITS>(std::make_integer_sequence<int, OB>{}, S, Up, inv, p, grp, group, go);
   if (!ok) return;
 #pragma unroll
   for (int i = 0; i < QNI; ++i) {
@@ -311,10 +330,9 @@ kronq_status quantize_split(cudaStream_t st, const kronq_opts &o, float *W,
   w += al(static_cast<size_t>(d_out) * m * 4);
   const size_t rest = ws_bytes - (static_cast<size_t>(w - static_cast<uint8_t *>(ws)));
   const int64_t ldq = o.bits * d_in / 32, lds = d_in / o.group;
-  if (cudaMemcpy2DAsync(W1, static_cast<size_t>(h) * 4, W, static_cast<size_t>(d_in) * 4,
+  KQ_CUDA(cudaMemcpy2DAsync(W1, static_cast<size_t>(h) * 4, W, static_cast<size_t>(d_in) * 4,
                         static_cast<size_t>(h) * 4, static_cast<size_t>(d_out),
-                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return KRONQ_ERR_CUDA;
+                        cudaMemcpyDeviceToDevice, st));
   QuantView v1{W, d_in, F, d_in, codes, ldq, scales, zeros, lds, d_out, h};
   KQ_TRY(quantize_view(st, o, v1, w, rest, info));
   {  // W1 − Ŵ1
