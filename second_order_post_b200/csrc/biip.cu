@@ -163,22 +163,13 @@ __device__ __forceinline__ void fwht_reg(float (&r)[R]) {
       }
 }
 
-// Threads [0, blockDim.x) and __syncthreads: the default work split of the
-// shared-memory rounds below.
-struct WholeBlock {
-  __device__ int tid() const { return threadIdx.x; }
-  __device__ int count() const { return blockDim.x; }
-  __device__ void sync() const { __syncthreads(); }
-};
-
 // One radix-R round of a length-L Hadamard over n_vec vectors held in shared
 // memory (element j of vector v at X[vbase(v) + j*stride]): combines the R
 // elements a + i*h, i < R, for every a whose index bits h .. R*h-1 are clear.
-template <int R, class VB, class TG = WholeBlock>
-__device__ void fwht_round(float *X, int n_vec, int L, int h, int stride, VB vbase,
-                           TG tg = TG{}) {
+template <int R, class VB>
+__device__ void fwht_round(float *X, int n_vec, int L, int h, int stride, VB vbase) {
   const int groups = L / R;
-  for (int idx = tg.tid(); idx < groups * n_vec; idx += tg.count()) {
+  for (int idx = threadIdx.x; idx < groups * n_vec; idx += blockDim.x) {
     const int v = idx % n_vec, g = idx / n_vec;
     const int a = (g / h) * R * h + (g % h);
     float *x = X + vbase(v) + a * stride;
@@ -189,21 +180,20 @@ __device__ void fwht_round(float *X, int n_vec, int L, int h, int stride, VB vba
 #pragma unroll
     for (int i = 0; i < R; ++i) x[i * h * stride] = r[i];
   }
-  tg.sync();
+  __syncthreads();
 }
 
 // Remaining rounds of a length-L Hadamard whose distances below h are done.
-template <class VB, class TG = WholeBlock>
-__device__ void fwht_rest(float *X, int n_vec, int L, int h, int stride, VB vbase,
-                          TG tg = TG{}) {
+template <class VB>
+__device__ void fwht_rest(float *X, int n_vec, int L, int h, int stride, VB vbase) {
   while (h * 16 <= L) {
-    fwht_round<16>(X, n_vec, L, h, stride, vbase, tg);
+    fwht_round<16>(X, n_vec, L, h, stride, vbase);
     h *= 16;
   }
   const int rem = L / h;
-  if (rem == 2) fwht_round<2>(X, n_vec, L, h, stride, vbase, tg);
-  else if (rem == 4) fwht_round<4>(X, n_vec, L, h, stride, vbase, tg);
-  else if (rem == 8) fwht_round<8>(X, n_vec, L, h, stride, vbase, tg);
+  if (rem == 2) fwht_round<2>(X, n_vec, L, h, stride, vbase);
+  else if (rem == 4) fwht_round<4>(X, n_vec, L, h, stride, vbase);
+  else if (rem == 8) fwht_round<8>(X, n_vec, L, h, stride, vbase);
 }
 
 // ------------------------------------------------------------- row pass
@@ -333,194 +323,6 @@ __global__ void __launch_bounds__(512, 2) row_pass_kernel(RowP p) {
         o[a * m + b] = y;
       }
     }
-  }
-}
-
-// ------------------------------------------------------------- pipelined row pass
-// Persistent form of the row pass for fp32 units (one unit = one chunk of
-// L*m contiguous columns of one row) with a column-side Q_m of 4 <= m <= 32,
-// m % 4 == 0. Each CTA walks the units blockIdx.x, blockIdx.x + gridDim.x, ...
-// with two shared-memory buffers: one producer lane moves units in and out by
-// bulk copies (cp.async.bulk, no multicast) while the compute warps transform
-// the other buffer in place. All waits are bounded.
-// (16 warps: registers are handed out to warps in groups of four, so a
-// 17-warp CTA would be charged for 20)
-constexpr int RPC = 480;         // compute threads
-constexpr int RPT = RPC + 32;    // + one producer warp
-
-struct ComputeGroup {
-  __device__ int tid() const { return threadIdx.x; }
-  __device__ int count() const { return RPC; }
-  __device__ void sync() const { asm volatile("bar.sync 1, %0;" ::"n"(RPC) : "memory"); }
-};
-
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
-                                          uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
-      "%2, [%3];" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// First Hadamard round (radix R0 over index bits below R0) fused with the
-// input factors norm * cr[row] * cc[col], in place in shared memory.
-template <int R0>
-__device__ void pipe_first_round(float *X, const RowP &p, float rf, int64_t c0) {
-  const int m = p.m, groups = p.L / R0;
-  for (int idx = threadIdx.x; idx < groups * m; idx += RPC) {
-    const int b = idx % m, g = idx / m;
-    float r[R0];
-#pragma unroll
-    for (int i = 0; i < R0; ++i) {
-      const int e = (g * R0 + i) * m + b;
-      float v = X[e] * rf;
-      if (p.cc) v *= __ldg(p.cc + c0 + e);
-      r[i] = v;
-    }
-    fwht_reg<R0>(r);
-#pragma unroll
-    for (int i = 0; i < R0; ++i) X[(g * R0 + i) * m + b] = r[i];
-  }
-  ComputeGroup{}.sync();
-}
-
-__global__ void __launch_bounds__(RPT, 1)
-    row_pass_pipe_kernel(RowP p, int64_t units, int chunk_pad, int32_t *info) {
-  extern __shared__ __align__(128) float rp_smem[];
-  __shared__ uint64_t full[2], done[2];
-  __shared__ int abort_flag, quiet_flag;
-  const int m = p.m, L = p.L, chunk = L * m;
-  const uint32_t bytes = static_cast<uint32_t>(chunk) * 4u;
-  auto buf = [&](int s) { return rp_smem + s * chunk_pad; };
-  if (threadIdx.x == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(&done[0], RPC);
-    mbar_init(&done[1], RPC);
-    abort_flag = 0;
-    quiet_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  const int64_t first = blockIdx.x, stride = gridDim.x;
-  const int64_t K = first < units ? (units - 1 - first) / stride + 1 : 0;
-  auto unit_row = [&](int64_t k) { return (first + k * stride) / p.chunks; };
-  auto unit_c0 = [&](int64_t k) { return ((first + k * stride) % p.chunks) * int64_t(chunk); };
-  if (threadIdx.x >= RPC) {
-    // ---- producer
-    if (threadIdx.x != RPC) return;
-    const float *in = static_cast<const float *>(p.in);
-    auto load = [&](int64_t k) {
-      const int s = static_cast<int>(k & 1);
-      mbar_expect_tx(&full[s], bytes);
-      bulk_load(buf(s), in + unit_row(k) * p.ld_in + unit_c0(k), bytes, &full[s]);
-    };
-    int64_t consumed = 0, issued = 0;
-    bool ok = true;
-    if (K > 0) {
-      load(0);
-      issued = 1;
-    }
-    for (int64_t k = 0; k < K; ++k) {
-      const int s = static_cast<int>(k & 1);
-      if (k + 1 < K) {
-        bulk_wait_read_all();  // the store of unit k-1 has left buffer s^1
-        load(k + 1);
-        issued = k + 2;
-      }
-      if (!mbar_wait(&done[s], static_cast<uint32_t>((k >> 1) & 1), &abort_flag)) {
-        ok = false;
-        break;
-      }
-      consumed = k + 1;
-      bulk_store(p.out + unit_row(k) * p.ld_out + unit_c0(k), buf(s), bytes);
-      bulk_commit();
-    }
-    if (!ok) {
-      report(info, KRONQ_ERR_TIMEOUT);
-      // let the loads still in flight land before the CTA leaves
-      for (int64_t k = consumed; k < issued; ++k)
-        mbar_wait(&full[k & 1], static_cast<uint32_t>((k >> 1) & 1), &quiet_flag);
-    }
-    bulk_wait_all();
-    return;
-  }
-  // ---- compute warps
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float q[32];
-#pragma unroll
-  for (int k = 0; k < 32; ++k) q[k] = (lane < m && k < m) ? p.Q[lane * m + k] : 0.f;
-  for (int64_t k = 0; k < K; ++k) {
-    const int s = static_cast<int>(k & 1);
-    if (!mbar_wait(&full[s], static_cast<uint32_t>((k >> 1) & 1), &abort_flag)) {
-      if (threadIdx.x == 0) report(info, KRONQ_ERR_TIMEOUT);
-      break;
-    }
-    float *X = buf(s);
-    const int64_t row = unit_row(k), c0 = unit_c0(k);
-    const float rf = p.norm * (p.cr ? p.cr[row] : 1.f);
-    int h;
-    if (L >= 16) {
-      pipe_first_round<16>(X, p, rf, c0);
-      h = 16;
-    } else if (L == 8) {
-      pipe_first_round<8>(X, p, rf, c0);
-      h = 8;
-    } else if (L == 4) {
-      pipe_first_round<4>(X, p, rf, c0);
-      h = 4;
-    } else if (L == 2) {
-      pipe_first_round<2>(X, p, rf, c0);
-      h = 2;
-    } else {
-      pipe_first_round<1>(X, p, rf, c0);
-      h = 1;
-    }
-    fwht_rest(X, m, L, h, m, [](int v) { return v; }, ComputeGroup{});
-    // Q_m over each group of m contiguous values, in place: a warp reads both
-    // of its groups completely before it writes them
-    for (int a = 2 * warp; a < L; a += 2 * (RPC / 32)) {
-      const bool two = a + 1 < L;
-      float4 *x0 = reinterpret_cast<float4 *>(X + a * m);
-      float4 *x1 = reinterpret_cast<float4 *>(X + (two ? a + 1 : a) * m);
-      float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-      for (int k4 = 0; k4 < 8; ++k4) {
-        if (4 * k4 < m) {
-          const float4 u = x0[k4], v = x1[k4];
-          y0 = fmaf(q[4 * k4], u.x, y0);
-          y0 = fmaf(q[4 * k4 + 1], u.y, y0);
-          y0 = fmaf(q[4 * k4 + 2], u.z, y0);
-          y0 = fmaf(q[4 * k4 + 3], u.w, y0);
-          y1 = fmaf(q[4 * k4], v.x, y1);
-          y1 = fmaf(q[4 * k4 + 1], v.y, y1);
-          y1 = fmaf(q[4 * k4 + 2], v.z, y1);
-          y1 = fmaf(q[4 * k4 + 3], v.w, y1);
-        }
-      }
-      __syncwarp();
-      if (lane < m) {
-        X[a * m + lane] = y0;
-        if (two) X[(a + 1) * m + lane] = y1;
-      }
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&done[s]);
   }
 }
 
@@ -795,7 +597,7 @@ kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
 kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in,
                     float *out, int64_t ld_out, int64_t R, int64_t C,
                     const SideRot &sr, const SideRot &sc, const float *cr,
-                    const float *cc, int32_t *info) {
+                    const float *cc) {
   const int64_t had_r = sr.rot ? sr.had : 1, m_r = sr.rot ? sr.m : 1;
   const int64_t had_c = sc.rot ? sc.had : 1, m_c = sc.rot ? sc.m : 1;
   // ---- row pass over chunks of Lc * m_c contiguous columns
@@ -835,33 +637,7 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
       p.m = static_cast<int>(chunk);
       p.Q = nullptr;
     }
-    const bool pipe = !in_bf16 && p.Q != nullptr && p.m >= 4 && p.m <= 32 &&
-                      p.m % 4 == 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 &&
-                      reinterpret_cast<uintptr_t>(out) % 16 == 0 && ld_in % 4 == 0 &&
-                      ld_out % 4 == 0 && chunk % 4 == 0;
-    if (pipe) {
-      static int sms = 0;
-      if (sms == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            sms <= 0)
-          return KRONQ_ERR_CUDA;
-      }
-      const int chunk_pad = static_cast<int>((chunk + 31) / 32 * 32);
-      const size_t pipe_smem = 2 * static_cast<size_t>(chunk_pad) * 4;
-      static bool pipe_attr = false;
-      if (!pipe_attr) {
-        KQ_CUDA(cudaFuncSetAttribute(row_pass_pipe_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 2 * ROW_CHUNK_MAX * 4));
-        pipe_attr = true;
-      }
-      const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(blocks, sms));
-      row_pass_pipe_kernel<<<grid, RPT, pipe_smem, st>>>(p, blocks, chunk_pad, info);
-    } else {
-      row_pass_kernel<<<static_cast<unsigned>(blocks), 512, smem, st>>>(p);
-    }
+    row_pass_kernel<<<static_cast<unsigned>(blocks), 512, smem, st>>>(p);
     KQ_CHECK_LAUNCH();
   }
   // ---- column-side Hadamard bits beyond the chunk
@@ -938,10 +714,10 @@ kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
   SideRot rx{d_in, o.rot_in.had, o.rot_in.m, rot_x, Qx};
   SideRot rg{d_out, o.rot_out.had, o.rot_out.m, rot_g, Qg};
   // W' = U_G (S_G W S_X) U_Xᵀ: rows use the output side, columns the input side
-  KQ_TRY(rotate(st, W, w_bf16, d_in, W_rot, d_in, d_out, d_in, rg, rx, fgw, fxw, info));
+  KQ_TRY(rotate(st, W, w_bf16, d_in, W_rot, d_in, d_out, d_in, rg, rx, fgw, fxw));
   // H_X' = U_X S_X^-1 H_X S_X^-1 U_Xᵀ, H_G' likewise (in place)
-  KQ_TRY(rotate(st, H_X, false, d_in, H_X, d_in, d_in, d_in, rx, rx, fxh, fxh, info));
-  KQ_TRY(rotate(st, H_G, false, d_out, H_G, d_out, d_out, d_out, rg, rg, fgh, fgh, info));
+  KQ_TRY(rotate(st, H_X, false, d_in, H_X, d_in, d_in, d_in, rx, rx, fxh, fxh));
+  KQ_TRY(rotate(st, H_G, false, d_out, H_G, d_out, d_out, d_out, rg, rg, fgh, fgh));
   return KRONQ_OK;
 }
 

@@ -620,6 +620,98 @@ bool same_operand(const GemmArgs &g) {
   return g.A == g.B && g.a_mn == g.b_mn && g.lda == g.ldb && g.M == g.N;
 }
 
+// ------------------------------------------------------------- small products
+// The small products at the bottom of the Cholesky recursion (128 .. 256 on a
+// side) sit one after another on its critical path, where a tensor-core
+// launch costs its pipeline fill and TMEM set-up for a few k-steps of work.
+// These run on the CUDA cores instead: plain fp32 FMA (exact products), one
+// 32 x 32 tile of C per CTA, the tile's A and B panels staged in shared
+// memory KC columns of k at a time with every load of a stage in flight at
+// once. The zero blocks of triangular operands are skipped like the tensor
+// kernel does, at this tile's granularity.
+constexpr int ST = 32;                 // tile edge
+constexpr int SKC = 128;               // k per shared-memory stage
+constexpr int STHREADS = 256;          // 16 x 16 threads, 2 x 2 outputs each
+constexpr int64_t kSmallMaxWork = int64_t(1) << 24;  // M*N*K at most (256^3)
+
+__global__ void __launch_bounds__(STHREADS)
+    small_gemm_kernel(GemmArgs g, int tiles_n) {
+  __shared__ __align__(16) float As[SKC][ST + 2];  // As[k][i]
+  __shared__ __align__(16) float Bs[SKC][ST + 2];  // Bs[k][j]
+  const int bm = blockIdx.x / tiles_n, bn = blockIdx.x % tiles_n;
+  if (g.upper_tiles_only && bm > bn) return;
+  const int64_t m0 = int64_t(bm) * ST, n0 = int64_t(bn) * ST;
+  int64_t kb = 0, ke = g.K;
+  if (g.kflags & KR_A_UPPER) kb = kq_max(kb, m0);
+  if (g.kflags & KR_B_UPPER) kb = kq_max(kb, n0);
+  if (g.kflags & KR_B_LOWER) ke = kq_min(ke, n0 + ST);
+  const int t = threadIdx.x, tx = t % 16, ty = t / 16;
+  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  for (int64_t k0 = kb; k0 < ke; k0 += SKC) {
+    const int kc = static_cast<int>(kq_min<int64_t>(SKC, ke - k0));
+    // stage: element e of the 32 x SKC panel; K-major operands are read along
+    // k (consecutive threads, consecutive k), MN-major ones along i / j
+    float va[ST * SKC / STHREADS], vb[ST * SKC / STHREADS];
+#pragma unroll
+    for (int u = 0; u < ST * SKC / STHREADS; ++u) {
+      const int e = t + u * STHREADS;
+      int i, kk;
+      if (g.a_mn) { kk = e / ST; i = e % ST; } else { i = e / SKC; kk = e % SKC; }
+      const int64_t gi = m0 + i, gk = k0 + kk;
+      va[u] = (gi < g.M && kk < kc)
+                  ? (g.a_mn ? g.A[gk * g.lda + gi] : g.A[gi * g.lda + gk])
+                  : 0.f;
+      int j, kj;
+      if (g.b_mn) { kj = e / ST; j = e % ST; } else { j = e / SKC; kj = e % SKC; }
+      const int64_t gj = n0 + j, gkb = k0 + kj;
+      vb[u] = (gj < g.N && kj < kc)
+                  ? (g.b_mn ? g.B[gkb * g.ldb + gj] : g.B[gj * g.ldb + gkb])
+                  : 0.f;
+    }
+    __syncthreads();  // the previous stage's readers are done
+#pragma unroll
+    for (int u = 0; u < ST * SKC / STHREADS; ++u) {
+      const int e = t + u * STHREADS;
+      if (g.a_mn) As[e / ST][e % ST] = va[u]; else As[e % SKC][e / SKC] = va[u];
+      if (g.b_mn) Bs[e / ST][e % ST] = vb[u]; else Bs[e % SKC][e / SKC] = vb[u];
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kc; ++kk) {
+      const float2 a = *reinterpret_cast<const float2 *>(&As[kk][2 * ty]);
+      const float2 b = *reinterpret_cast<const float2 *>(&Bs[kk][2 * tx]);
+      acc[0][0] = fmaf(a.x, b.x, acc[0][0]);
+      acc[0][1] = fmaf(a.x, b.y, acc[0][1]);
+      acc[1][0] = fmaf(a.y, b.x, acc[1][0]);
+      acc[1][1] = fmaf(a.y, b.y, acc[1][1]);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int64_t i = m0 + 2 * ty + r;
+    if (i >= g.M) continue;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int64_t j = n0 + 2 * tx + c;
+      if (j >= g.N) continue;
+      float *cp = g.C + i * g.ldc + j;
+      const float v = g.alpha * acc[r][c];
+      *cp = g.beta != 0.f ? fmaf(g.beta, *cp, v) : v;
+    }
+  }
+}
+
+bool small_ok(const GemmArgs &g) { return g.M * g.N * g.K <= kSmallMaxWork; }
+
+kronq_status launch_small(cudaStream_t st, const GemmArgs &g) {
+  const int64_t tm = ceil_div(g.M, ST), tn = ceil_div(g.N, ST);
+  if (tm * tn > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+  small_gemm_kernel<<<static_cast<unsigned>(tm * tn), STHREADS, 0, st>>>(
+      g, static_cast<int>(tn));
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
 }  // namespace
 
 kronq_status gemm_tf32x3(cudaStream_t st, const GemmArgs &g, int32_t *info) {
@@ -640,6 +732,7 @@ kronq_status gemm_f32(cudaStream_t st, const GemmArgs &g, void *scratch,
   if (g.M < 0 || g.N < 0 || g.K < 0) return KRONQ_ERR_INVALID_ARG;
   if (g.M == 0 || g.N == 0) return KRONQ_OK;
   if (g.upper_tiles_only && g.M != g.N) return KRONQ_ERR_INVALID_ARG;
+  if (small_ok(g)) return launch_small(st, g);
   const bool f16 = scratch && g.K > 0 && wide_ok(g) && g.M * g.N * g.K >= kF16MinWork &&
                    scratch_bytes >= gemm_scratch_bytes(g.M, g.N, g.K);
   if (!f16) return gemm_tf32x3(st, g, info);
