@@ -269,7 +269,7 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
                               double *loss_dev, void *ws, size_t ws_bytes);
 
 /*
- * fp32-accurate dense product on the tensor cores (the contraction behind the
+ * fp32-accurate dense product, on the tensor cores (the contraction behind the
  * Cholesky recursion, the OBS trailing updates and the layer loss; the pages
  * name no such routine): C = alpha * A * B^T + beta * C with row-major
  * operands on the device,
@@ -281,7 +281,9 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
  * products when ws holds kronq_gemm_f32_workspace_bytes(M, N, K) bytes
  * (device, 256-byte aligned, busy until the product completes on the stream),
  * fp16 parts of the operand rows scaled by powers of two. ws may be NULL.
- * Pointers 16-byte aligned, pitches multiples of 4 elements; M, N, K >= 0.
+ * Small products (M * N * K <= 2^24) skip the split and run as plain fp32
+ * FMA on the CUDA cores, where a tensor-core pipeline costs more to set up
+ * than it saves. Pointers 16-byte aligned, pitches multiples of 4 elements; M, N, K >= 0.
  * C must not overlap A or B. INVALID_ARG for negative sizes or null
  * pointers, UNSUPPORTED for misaligned operands, TIMEOUT in *info_dev
  * (nonzero) if a pipeline wait ran out.

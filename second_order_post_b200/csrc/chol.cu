@@ -10,11 +10,12 @@
 //     A  <- A - V Vᵀ                (R11 R11ᵀ)
 //     U11 = inv_chol(A)             (recursive)
 //     U12 = -U11 (V U22)
-// All off-diagonal work runs as fp32-accurate 3xTF32 tcgen05 GEMMs that skip
-// the zero blocks of the triangular operands; 128x128 diagonal leaves are
-// factored and inverted in registers by one CTA. λ = damp_rel * mean(diag H) is added
-// by each leaf to its own diagonal (the updates never touch λ, so this equals
-// damping H up front).
+// All off-diagonal work runs through gemm_f32, which skips the zero blocks of
+// the triangular operands: fp16-split tcgen05 products for the large nodes,
+// 3xTF32 for the mid-size ones, plain fp32 FMA on the CUDA cores for the
+// smallest. 128x128 diagonal leaves are factored and inverted in registers by
+// one CTA. λ = damp_rel * mean(diag H) is added by each leaf to its own
+// diagonal (the updates never touch λ, so this equals damping H up front).
 #include <mutex>
 
 #include "kernels.cuh"

@@ -44,6 +44,15 @@ def test_status_strings(K):
     assert K.kronq_status_string(99) == "unknown status"
 
 
+def test_last_cuda_error_and_error_text(K):
+    """No CUDA call has failed in this process: the diagnostic reads
+    "no error", and a KRONQ_ERR_CUDA exception carries the CUDA text."""
+    assert K._lib.kronq_last_cuda_error().decode() == "no error"
+    e = K.KronqError("kronq_x", K.KRONQ_ERR_CUDA)
+    assert str(e).endswith("no error (status 6)")
+    assert "no error" not in str(K.KronqError("kronq_x", K.KRONQ_ERR_INVALID_ARG))
+
+
 def test_invalid_args_rejected_before_device(K):
     lib = K._lib
     nullp = ctypes.c_void_p(0)
