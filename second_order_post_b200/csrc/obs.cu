@@ -4,14 +4,14 @@
 // W2/W3/W4 with 128-column groups].
 //
 // Per 128-column block j0 (one launch of obs_block_kernel): eight lanes share
-// one row, lane p of the group holding the columns 8i + p (i < 16) in
+// one row, lane p of the eight holding the columns 8i + p (i < 16) in
 // registers, so that every lane has about the same number of updates left at
 // any column. U[j0:j0+128, j0:j0+128] sits in shared memory, permuted so that
 // each lane's columns of a U row are contiguous. The sweep over the block's
 // 128 columns is unrolled, so every register index is a compile-time
 // constant. For each column j: group (scale, zero) at a group start,
-// q = clamp(rint(w/scale)+zero), err = (w - w_hat)/U[j][j] (all lanes of
-// the row's group compute them from the owner's weight), w_k -= err * U[j][k] for
+// q = clamp(rint(w/scale)+zero), err = (w - w_hat)/U[j][j] (the row's eight
+// lanes all compute them from the owner's weight), w_k -= err * U[j][k] for
 // the block's k > j. The errors go to E; the columns right of the block are
 // updated lazily by 3xTF32 GEMMs: within a super-block of S columns after
 // every block (W[:, blk_end:sb_end] -= E_blk U[blk, blk_end:sb_end]), and
@@ -57,7 +57,7 @@ struct GroupOut {
 // Column J of the block (every register index is a compile-time constant).
 template <int BITS, int J>
 __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
-                                           const float *inv, int p, int grp,
+                                           const float *inv, int p, int lane0,
                                            int group, const GroupOut &go) {
   constexpr int io = J / QLPR, po = J % QLPR;
   constexpr float maxq = static_cast<float>((1 << BITS) - 1);
@@ -95,7 +95,7 @@ __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
   }
   const float4 *u4 = reinterpret_cast<const float4 *>(Up + J * QUROW + p * QUP);
   const float iu = inv[J];
-  const float wj = __shfl_sync(0xffffffffu, S.w[io], grp | po);
+  const float wj = __shfl_sync(0xffffffffu, S.w[io], lane0 | po);
   // w/scale as a product with the group's reciprocal: it can differ from
   // the quotient only within an ulp of a rounding tie
   const float q = fminf(fmaxf(rintf(wj * S.rscale) + S.zero, 0.f), maxq);
@@ -115,8 +115,8 @@ __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
     for (int c = 0; c < 4; ++c) {
       const int i = 4 * a + c;
       if (i == io) {
-        // the column itself: the owner keeps w_hat and the error, the lanes
-        // right of it in the row's group update their column of the same i
+        // the column itself: the owner keeps w_hat and the error, the row's
+        // lanes right of it update their column of the same i
         if (p > po) S.w[i] = fmaf(-e, uu[c], S.w[i]);
         else if (p == po) {
           S.w[i] = wh;
@@ -132,9 +132,9 @@ __device__ __forceinline__ void obs_column(SweepState<BITS> &S, const float *Up,
 template <int BITS, int... J>
 __device__ __forceinline__ void obs_sweep(std::integer_sequence<int, J...>,
                                           SweepState<BITS> &S, const float *Up,
-                                          const float *inv, int p, int grp, int group,
+                                          const float *inv, int p, int lane0, int group,
                                           const GroupOut &go) {
-  (obs_column<BITS, J>(S, Up, inv, p, grp, group, go), ...);
+  (obs_column<BITS, J>(S, Up, inv, p, lane0, group, go), ...);
 }
 
 // One 128-column block for OROWS rows per CTA (32 / QLPR rows per warp).
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(OTHREADS)
   extern __shared__ __align__(16) float Up[];  // Up[j][p][i] = U[j][QLPR*i + p]
   float *inv = Up + OB * QUROW;                // 1/U[j][j]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = lane & (QLPR - 1), grp = lane & ~(QLPR - 1);
+  const int p = lane & (QLPR - 1), lane0 = lane & ~(QLPR - 1);
   const int64_t row = int64_t(blockIdx.x) * OROWS + warp * (32 / QLPR) + lane / QLPR;
   const bool ok = row < d_out;
   SweepState<BITS> S;
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(OTHREADS)
   __syncthreads();
   const GroupOut go{scales + row * ngroups, zeros + row * ngroups, j0 / group,
                     p == 0 && ok};
-  obs_sweep<BITS>(std::make_integer_sequence<int, OB>{}, S, Up, inv, p, grp, group, go);
+  obs_sweep<BITS>(std::make_integer_sequence<int, OB>{}, S, Up, inv, p, lane0, group, go);
   if (!ok) return;
 #pragma unroll
   for (int i = 0; i < QNI; ++i) {
