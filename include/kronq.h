@@ -169,10 +169,13 @@ typedef enum {
  * and a 16-byte aligned A; otherwise KRONQ_ERR_UNSUPPORTED. n == 0 scales H by
  * beta. Symmetric in its result; the two triangles are written from the same
  * accumulator tile, so they are bitwise equal.
+ * info_dev: KRONQ_ERR_TIMEOUT when a pipeline wait of the tensor-core path
+ * ran out (H is then incomplete and must not be used).
  */
 kronq_status kronq_accum_cov(kronq_stream_t stream, const void *A,
                              kronq_dtype dtype, int64_t n, int64_t d,
-                             int64_t lda, float alpha, float beta, float *H);
+                             int64_t lda, float alpha, float beta, float *H,
+                             int32_t *info_dev);
 
 /*
  * Step 2 — sublayer sensitivity [wmrh §三, §六; aimodeling].
@@ -220,6 +223,8 @@ kronq_status kronq_biip(kronq_stream_t stream, const kronq_opts *opts,
  *   earlier in the same call.
  * - Calls that overlap on the GPU (other streams, other host threads) race
  *   on the array. Serialise them.
+ * - The cached address belongs to the device's current CUDA context; do not
+ *   keep using the library across cudaDeviceReset in the same process.
  * - Sizes whose scratch would not fit return KRONQ_ERR_UNSUPPORTED. Every
  *   size that kronq_biip accepts (d <= 65536, m <= 256) fits.
  */
@@ -236,7 +241,13 @@ kronq_status kronq_biip_noalloc(kronq_stream_t stream, const kronq_opts *opts,
  * triangular with U^T U = (H + lambda I)^-1, lambda = damp_rel * mean(diag H),
  * strict lower triangle set to 0. Computed as H + lambda I = R R^T (R upper,
  * reverse-order Cholesky) and U = R^-1, in fp32 with 3xTF32 tensor-core
- * trailing updates. Requires d % 128 == 0. info: NOT_PD with the column.
+ * trailing updates. Requires d % 128 == 0. info: NOT_PD with the column;
+ * NONFINITE when the mean of the diagonal is not finite.
+ * Shared state: the recursion forks onto CUDA streams and events that the
+ * library creates once per device and keeps. Calls on one device from several
+ * host threads are therefore serialised: each call holds a per-device lock
+ * while it enqueues, and its work queues behind the previous call's work on
+ * those internal streams.
  */
 kronq_status kronq_chol_inv(kronq_stream_t stream, float *H, int64_t d,
                             float damp_rel, void *ws, size_t ws_bytes,
@@ -261,12 +272,27 @@ kronq_status kronq_quantize_sublayer(kronq_stream_t stream,
 /*
  * Measurement — the Kronecker-factored layer loss [aimodeling: H ≈ H_X ⊗ H_G;
  * wmrh §二]: *loss_dev = tr(H_G dW H_X dW^T) with dW = W_ref - W_hat, summed in
- * fp64 over fp32 products (3xTF32 tensor-core GEMMs). d_in, d_out % 128 == 0.
+ * fp64 over fp32 products (fp32-accurate tensor-core GEMMs). d_in, d_out % 128
+ * == 0. ws: kronq_workspace_bytes(KRONQ_WS_LOSS, ...). info_dev: TIMEOUT when
+ * a GEMM pipeline wait ran out (the loss is then not valid).
  */
 kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
                               const float *W_hat, const float *H_X,
                               const float *H_G, int64_t d_out, int64_t d_in,
-                              double *loss_dev, void *ws, size_t ws_bytes);
+                              double *loss_dev, void *ws, size_t ws_bytes,
+                              int32_t *info_dev);
+
+/*
+ * Diagnostics (no counterpart on the pages): exercises the library's bounded
+ * device wait. One kernel waits on a shared-memory barrier that nothing
+ * completes, through the same wait routine the tensor-core pipelines use,
+ * with a limit of limit_ns (1 .. 1e9 ns) instead of their 4 s. The wait gives
+ * up, the kernel writes KRONQ_ERR_TIMEOUT to *info_dev and returns; the CUDA
+ * context stays usable. Lets a caller check, without any fault, that a wait
+ * which runs out is reported rather than hanging.
+ */
+kronq_status kronq_selftest_timeout(kronq_stream_t stream, uint64_t limit_ns,
+                                    int32_t *info_dev);
 
 /*
  * fp32-accurate dense product, on the tensor cores (the contraction behind the

@@ -41,18 +41,20 @@ const char *kronq_status_string(kronq_status s) {
 
 kronq_status kronq_accum_cov(kronq_stream_t stream, const void *A,
                              kronq_dtype dtype, int64_t n, int64_t d,
-                             int64_t lda, float alpha, float beta, float *H) {
-  if (!H || d <= 0 || n < 0 || lda < d || (n > 0 && !A))
+                             int64_t lda, float alpha, float beta, float *H,
+                             int32_t *info_dev) {
+  if (!H || !info_dev || d <= 0 || n < 0 || lda < d || (n > 0 && !A))
     return KRONQ_ERR_INVALID_ARG;
   if (dtype != KRONQ_F32 && dtype != KRONQ_BF16) return KRONQ_ERR_INVALID_ARG;
   if (d > (int64_t(1) << 20) || n > (int64_t(1) << 31)) return KRONQ_ERR_UNSUPPORTED;
+  if (dtype == KRONQ_BF16 && (d % 128 || lda % 8 || !aligned(A, 16)))
+    return KRONQ_ERR_UNSUPPORTED;
   KQ_TRY(require_sm100());
   cudaStream_t st = as_stream(stream);
-  if (dtype == KRONQ_BF16) {
-    if (d % 128 || lda % 8 || !aligned(A, 16)) return KRONQ_ERR_UNSUPPORTED;
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  if (dtype == KRONQ_BF16)
     return cov_bf16(st, static_cast<const __nv_bfloat16 *>(A), n, d, lda, alpha,
-                    beta, H);
-  }
+                    beta, H, info_dev);
   return cov_f32(st, static_cast<const float *>(A), n, d, lda, alpha, beta, H);
 }
 
@@ -196,9 +198,10 @@ kronq_status kronq_quantize_split(kronq_stream_t stream, const kronq_opts *opts,
 kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
                               const float *W_hat, const float *H_X,
                               const float *H_G, int64_t d_out, int64_t d_in,
-                              double *loss_dev, void *ws, size_t ws_bytes) {
-  if (!W_ref || !W_hat || !H_X || !H_G || !loss_dev || !ws || d_out <= 0 ||
-      d_in <= 0)
+                              double *loss_dev, void *ws, size_t ws_bytes,
+                              int32_t *info_dev) {
+  if (!W_ref || !W_hat || !H_X || !H_G || !loss_dev || !ws || !info_dev ||
+      d_out <= 0 || d_in <= 0)
     return KRONQ_ERR_INVALID_ARG;
   if (d_in % 128 || d_out % 128) return KRONQ_ERR_UNSUPPORTED;
   if (!aligned(ws, 256) || !aligned(W_ref, 16) || !aligned(W_hat, 16) ||
@@ -206,8 +209,20 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
     return KRONQ_ERR_INVALID_ARG;
   if (ws_bytes < loss_ws_bytes(d_out, d_in)) return KRONQ_ERR_INVALID_ARG;
   KQ_TRY(require_sm100());
-  return layer_loss(as_stream(stream), W_ref, W_hat, H_X, H_G, d_out, d_in,
-                    loss_dev, ws, ws_bytes);
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return layer_loss(st, W_ref, W_hat, H_X, H_G, d_out, d_in, loss_dev, ws,
+                    ws_bytes, info_dev);
+}
+
+kronq_status kronq_selftest_timeout(kronq_stream_t stream, uint64_t limit_ns,
+                                    int32_t *info_dev) {
+  if (!info_dev || limit_ns == 0 || limit_ns > kSelftestMaxNs)
+    return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return launch_selftest_timeout(st, limit_ns, info_dev);
 }
 
 kronq_status kronq_gemm_f32(kronq_stream_t stream, int64_t M, int64_t N,

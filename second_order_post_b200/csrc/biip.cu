@@ -549,17 +549,8 @@ constexpr int64_t MAX_A = 1024;           // Hadamard length of one strided pass
 // sees its independent vectors on a two-level outer index.
 kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
                             int64_t so, int64_t A, int64_t smid, int64_t inner) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(strided_fwht_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SLAB_FLOATS * 4) != cudaSuccess ||
-        cudaFuncSetAttribute(strided_fwht4_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SLAB_FLOATS * 4) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr_done = true;
-  }
+  KQ_TRY(smem_attr(strided_fwht_kernel, SLAB_FLOATS * 4));
+  KQ_TRY(smem_attr(strided_fwht4_kernel, SLAB_FLOATS * 4));
   if (A <= 1) return KRONQ_OK;
   const bool vec = reinterpret_cast<uintptr_t>(base) % 16 == 0 && so % 4 == 0 &&
                    smid % 4 == 0 && inner % 4 == 0;
@@ -620,13 +611,7 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
     p.Q = (sc.rot && m_c > 1) ? sc.Q : nullptr;
     p.chunks = C / chunk;
     size_t smem = static_cast<size_t>(chunk) * 4;
-    static bool attr_done = false;
-    if (!attr_done) {
-      KQ_CUDA(cudaFuncSetAttribute(row_pass_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ROW_CHUNK_MAX * 4));
-      attr_done = true;
-    }
+    KQ_TRY(smem_attr(row_pass_kernel, static_cast<int>(ROW_CHUNK_MAX * 4)));
     if (C % chunk) return KRONQ_ERR_UNSUPPORTED;
     const int64_t blocks = R * p.chunks;
     if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
@@ -649,13 +634,7 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
     const size_t smem =
         (static_cast<size_t>(m_r) * m_r + (m_r > 32 ? m_r * 64 : m_r * m_r)) * 4;
     if (smem > 227 * 1024) return KRONQ_ERR_UNSUPPORTED;
-    static bool attr_done = false;
-    if (!attr_done) {
-      KQ_CUDA(cudaFuncSetAttribute(rowq_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024));
-      attr_done = true;
-    }
+    KQ_TRY(smem_attr(rowq_kernel, 227 * 1024));
     const int64_t cols = m_r > 32 ? 64 : 256;
     dim3 grid(static_cast<unsigned>(ceil_div(C, cols)), static_cast<unsigned>(had_r));
     rowq_kernel<<<grid, 256, smem, st>>>(out, ld_out, C, static_cast<int>(m_r), sr.Q);

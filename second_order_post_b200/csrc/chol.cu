@@ -295,6 +295,10 @@ struct Ctx {
 // the next free SM ahead of the concurrent T products.
 struct CholStreams {
   bool ready = false;
+  // held by one call from its fork record to its last join: the fork and
+  // join events are shared by every call on the device, so two host threads
+  // must not interleave their records and waits
+  std::mutex call_mu;
   cudaStream_t main;
   cudaStream_t side[MAXD];
   cudaEvent_t ev_v[MAXD], ev_t[MAXD], fork, join_main, join_side[MAXD];
@@ -457,6 +461,7 @@ kronq_status chol_run(cudaStream_t st, float *H, int64_t d, float damp_rel,
   if (ws_bytes < need) return KRONQ_ERR_INVALID_ARG;
   CholStreams *cs = nullptr;
   KQ_TRY(chol_streams(&cs));
+  std::lock_guard<std::mutex> call_lock(cs->call_mu);
   uint8_t *w = static_cast<uint8_t *>(ws);
   Ctx c;
   c.st = cs->main;

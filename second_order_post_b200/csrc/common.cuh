@@ -46,6 +46,15 @@ kronq_status cuda_fail(cudaError_t e);
 // Device ordinal check: the library runs on sm_100 only.
 kronq_status require_sm100();
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device. The attribute belongs to the device context, so it is set once per
+// (device, kernel, size); thread-safe.
+kronq_status set_max_dyn_smem(const void *func, int bytes);
+template <class F>
+inline kronq_status smem_attr(F *func, int bytes) {
+  return set_max_dyn_smem(reinterpret_cast<const void *>(func), bytes);
+}
+
 // 2D tiled tensor map over a row-major fp32/bf16 matrix: inner extent `inner`
 // (contiguous), outer extent `outer`, row pitch `pitch_elems`, box
 // {box_inner, box_outer}, zero fill out of bounds. Swizzle: TMAP_SW128
@@ -66,6 +75,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Bounded device waits give up after this many nanoseconds of wall time and
 // report KRONQ_ERR_TIMEOUT instead of spinning forever.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// Upper bound of the wait limit kronq_selftest_timeout accepts.
+constexpr uint64_t kSelftestMaxNs = 1000000000ull;
 
 // ----------------------------------------------------------------- device side
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -134,16 +145,19 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 
 // Waits for the phase of `bar` with the given parity to complete. Returns
 // false (and leaves the barrier untouched) once *abort is set by another
-// thread or the wall-time limit passes; the caller then winds down. Between
-// checks the thread sleeps on the barrier for up to 0.5 ms.
+// thread or the wall-time limit `limit_ns` passes; the caller then winds
+// down. Between checks the thread sleeps on the barrier for up to 0.5 ms (1 us
+// under limits below 1 ms).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort) {
+                                          volatile int *abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint32_t nap = limit_ns < 1000000ull ? 1000u : 500000u;
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
+    if (mbar_try_wait_sleep(bar, parity, nap)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       return false;
     }

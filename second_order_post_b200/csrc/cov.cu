@@ -322,21 +322,15 @@ kronq_status scale_matrix(cudaStream_t st, float *H, int64_t n_elems, float beta
 
 kronq_status cov_bf16(cudaStream_t st, const __nv_bfloat16 *A, int64_t n,
                       int64_t d, int64_t lda, float alpha, float beta,
-                      float *H) {
+                      float *H, int32_t *info) {
   if (n == 0) return scale_matrix(st, H, d * d, beta);
   CUtensorMap tm;
   KQ_TRY(make_tmap_2d(&tm, A, true, d, n, lda, 64, CBK));
   const int64_t nt = ceil_div(d, CT);
   const int64_t tiles = nt * (nt + 1) / 2;
-  static bool attr_done = false;
-  if (!attr_done) {
-    KQ_CUDA(cudaFuncSetAttribute(cov_bf16_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CSMEM));
-    attr_done = true;
-  }
+  KQ_TRY(smem_attr(cov_bf16_kernel, CSMEM));
   cov_bf16_kernel<<<static_cast<unsigned>(tiles), CTHREADS, CSMEM, st>>>(
-      tm, n, d, alpha, beta, H, nullptr);
+      tm, n, d, alpha, beta, H, info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }

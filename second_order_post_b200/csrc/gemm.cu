@@ -428,12 +428,7 @@ kronq_status launch(cudaStream_t st, const GemmArgs &g, int32_t *info,
     for (int64_t bi = 0; bi < tm; ++bi) tiles += tn - upper_first<C>(bi);
   }
   if (tiles > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
-  static bool attr_done = false;
-  if (!attr_done) {
-    KQ_CUDA(cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM));
-    attr_done = true;
-  }
+  KQ_TRY(smem_attr(gemm_kernel<C>, C::SMEM));
   GemmP p;
   p.M = g.M; p.N = g.N; p.K = g.K;
   p.C = g.C; p.ldc = g.ldc;

@@ -44,7 +44,7 @@ size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 // ---------------------------------------------------------------- covariance
 kronq_status cov_bf16(cudaStream_t st, const __nv_bfloat16 *A, int64_t n,
                       int64_t d, int64_t lda, float alpha, float beta,
-                      float *H);
+                      float *H, int32_t *info);
 kronq_status cov_f32(cudaStream_t st, const float *A, int64_t n, int64_t d,
                      int64_t lda, float alpha, float beta, float *H);
 kronq_status scale_matrix(cudaStream_t st, float *H, int64_t n_elems,
@@ -54,6 +54,8 @@ kronq_status scale_matrix(cudaStream_t st, float *H, int64_t n_elems,
 kronq_status launch_sensitivity(cudaStream_t st, const float *hx, int64_t dx,
                                 const float *hg, int64_t dg, double *out);
 kronq_status launch_set_int(cudaStream_t st, int32_t *p, int32_t v);
+kronq_status launch_selftest_timeout(cudaStream_t st, uint64_t limit_ns,
+                                     int32_t *info);
 uint64_t launches();
 int last_cuda_error();
 
@@ -105,6 +107,6 @@ size_t loss_ws_bytes(int64_t d_out, int64_t d_in);
 kronq_status layer_loss(cudaStream_t st, const float *W_ref,
                         const float *W_hat, const float *H_X, const float *H_G,
                         int64_t d_out, int64_t d_in, double *loss, void *ws,
-                        size_t ws_bytes);
+                        size_t ws_bytes, int32_t *info);
 
 }  // namespace kronq

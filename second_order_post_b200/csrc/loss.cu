@@ -39,7 +39,8 @@ size_t loss_ws_bytes(int64_t d_out, int64_t d_in) {
 
 kronq_status layer_loss(cudaStream_t st, const float *W_ref, const float *W_hat,
                         const float *H_X, const float *H_G, int64_t d_out,
-                        int64_t d_in, double *loss, void *ws, size_t ws_bytes) {
+                        int64_t d_in, double *loss, void *ws, size_t ws_bytes,
+                        int32_t *info) {
   if (ws_bytes < loss_ws_bytes(d_out, d_in)) return KRONQ_ERR_INVALID_ARG;
   const size_t one = (static_cast<size_t>(d_out) * d_in * 4 + 255) / 256 * 256;
   uint8_t *w = static_cast<uint8_t *>(ws);
@@ -57,13 +58,13 @@ kronq_status layer_loss(cudaStream_t st, const float *W_ref, const float *W_hat,
   g.A = D; g.lda = d_in;
   g.B = H_X; g.ldb = d_in;
   g.C = P; g.ldc = d_in;
-  KQ_TRY(gemm_f32(st, g, scr, scr_bytes, nullptr));
+  KQ_TRY(gemm_f32(st, g, scr, scr_bytes, info));
   GemmArgs h;  // Q = H_G D
   h.M = d_out; h.N = d_in; h.K = d_out;
   h.A = H_G; h.lda = d_out;
   h.B = D; h.ldb = d_in; h.b_mn = true;
   h.C = Q; h.ldc = d_in;
-  KQ_TRY(gemm_f32(st, h, scr, scr_bytes, nullptr));
+  KQ_TRY(gemm_f32(st, h, scr, scr_bytes, info));
   KQ_CUDA(cudaMemsetAsync(loss, 0, sizeof(double), st));
   dot_kernel<<<blocks, 256, 0, st>>>(P, Q, n, loss);
   KQ_CHECK_LAUNCH();

@@ -3,6 +3,9 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
+#include <set>
+#include <tuple>
 
 #include "kernels.cuh"
 
@@ -35,6 +38,19 @@ __global__ void sensitivity_kernel(const float *hx, int64_t dx, const float *hg,
 }
 
 __global__ void set_int_kernel(int32_t *p, int32_t v) { *p = v; }
+
+// One thread waits, through the library's bounded mbarrier wait, on a barrier
+// that nothing ever completes: the wait must give up after limit_ns and the
+// kernel must report KRONQ_ERR_TIMEOUT and return.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns, int32_t *info) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait(&bar, 0, &abort_flag, limit_ns)) report(info, KRONQ_ERR_TIMEOUT);
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -69,20 +85,39 @@ int last_cuda_error() { return g_last_cuda.load(std::memory_order_relaxed); }
 
 uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
+namespace {
+constexpr int kMaxDev = 64;
+// per device: 0 = not checked yet, 1 = sm_100, 2 = another architecture
+std::atomic<int> g_arch_ok[kMaxDev];
+}  // namespace
+
 kronq_status require_sm100() {
   int dev = -1;
   KQ_CUDA(cudaGetDevice(&dev));
-  static int checked_dev = -1;
-  static bool ok = false;
-  if (checked_dev != dev) {
+  if (dev < 0 || dev >= kMaxDev) return KRONQ_ERR_UNSUPPORTED;
+  int state = g_arch_ok[dev].load(std::memory_order_acquire);
+  if (state == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return KRONQ_ERR_CUDA;
-    ok = (major == 10 && minor == 0);
-    checked_dev = dev;
+    state = (major == 10 && minor == 0) ? 1 : 2;
+    g_arch_ok[dev].store(state, std::memory_order_release);
   }
-  return ok ? KRONQ_OK : KRONQ_ERR_CUDA;
+  return state == 1 ? KRONQ_OK : KRONQ_ERR_CUDA;
+}
+
+kronq_status set_max_dyn_smem(const void *func, int bytes) {
+  int dev = -1;
+  KQ_CUDA(cudaGetDevice(&dev));
+  static std::mutex mu;
+  static std::set<std::tuple<int, const void *, int>> done;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(dev, func, bytes);
+  if (done.count(key)) return KRONQ_OK;
+  KQ_CUDA(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done.insert(key);
+  return KRONQ_OK;
 }
 
 kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
@@ -113,6 +148,13 @@ kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
 kronq_status launch_sensitivity(cudaStream_t st, const float *hx, int64_t dx,
                                 const float *hg, int64_t dg, double *out) {
   sensitivity_kernel<<<1, 1024, 0, st>>>(hx, dx, hg, dg, out);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
+kronq_status launch_selftest_timeout(cudaStream_t st, uint64_t limit_ns,
+                                     int32_t *info) {
+  selftest_timeout_kernel<<<1, 32, 0, st>>>(limit_ns, info);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }

@@ -239,17 +239,9 @@ kronq_status quantize_view(cudaStream_t st, const kronq_opts &o, const QuantView
   const size_t e_bytes = (static_cast<size_t>(d_out) * S * 4 + 255) / 256 * 256;
   void *scr = static_cast<uint8_t *>(ws) + e_bytes;
   const size_t scr_bytes = ws_bytes - e_bytes;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(obs_block_kernel<2>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, OSMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(obs_block_kernel<3>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, OSMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(obs_block_kernel<4>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, OSMEM) != cudaSuccess)
-      return KRONQ_ERR_CUDA;
-    attr_done = true;
-  }
+  KQ_TRY(smem_attr(obs_block_kernel<2>, OSMEM));
+  KQ_TRY(smem_attr(obs_block_kernel<3>, OSMEM));
+  KQ_TRY(smem_attr(obs_block_kernel<4>, OSMEM));
   auto block_kernel = o.bits == 2 ? obs_block_kernel<2>
                       : o.bits == 3 ? obs_block_kernel<3>
                                     : obs_block_kernel<4>;

@@ -60,7 +60,8 @@ class SublayerEngine:
         self.codes = torch.empty(d_out, bits * d_in // 32, dtype=torch.int32, device=dev)
         self.scales = torch.empty(d_out, ng, **f32)
         self.zeros = torch.empty(d_out, ng, dtype=torch.uint8, device=dev)
-        self.info = torch.zeros(3, dtype=torch.int32, device=dev)
+        # status words: cov X, cov G, BiIP, Cholesky, OBS
+        self.info = torch.zeros(5, dtype=torch.int32, device=dev)
         kinds = [K.KRONQ_WS_BIIP, K.KRONQ_WS_CHOL,
                  K.KRONQ_WS_QUANT_SPLIT if self.split else K.KRONQ_WS_QUANT]
         ws = max(K.kronq_workspace_bytes(k, d_out, d_in, self.opts) for k in kinds)
@@ -69,38 +70,40 @@ class SublayerEngine:
         self.ws = torch.empty((ws + 255) // 256 * 256, dtype=torch.uint8, device=dev)
 
     def covariances(self, X, G, stream=None):
-        K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, stream)
-        K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, stream)
+        K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, self.info[0:1], stream)
+        K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, self.info[1:2], stream)
 
     def run(self, W, X, G, stream=None, mark=None) -> QuantResult:
         """Enqueue the whole sublayer quantization (no host synchronisation).
         ``mark(name)``, if given, is called after each step is enqueued (the
         benchmark records a CUDA event there)."""
         mark = mark or (lambda name: None)
-        K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, stream)
+        K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, self.info[0:1],
+                          stream)
         mark("cov_x")
-        K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, stream)
+        K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, self.info[1:2],
+                          stream)
         mark("cov_g")
         K.kronq_sensitivity(self.H_X, self.H_G, self.sens, stream)
         K.kronq_biip(self.opts, W, self.W_rot, self.H_X, self.H_G, self.s_x,
-                     self.s_g, self.ws, self.info[0:1], stream)
+                     self.s_g, self.ws, self.info[2:3], stream)
         mark("biip")
         if self.W_ref is not None:
             self.W_ref.copy_(self.W_rot)
         if self.split:
             K.kronq_chol_split(self.H_X, self.opts.damp_rel, self.ws,
-                               self.info[1:2], stream)
+                               self.info[3:4], stream)
             mark("chol")
             K.kronq_quantize_split(self.opts, self.W_rot, self.H_X, self.codes,
                                    self.scales, self.zeros, self.ws,
-                                   self.info[2:3], stream)
+                                   self.info[4:5], stream)
         else:
-            K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[1:2],
+            K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[3:4],
                              stream)
             mark("chol")
             K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, self.codes,
                                       self.scales, self.zeros, self.ws,
-                                      self.info[2:3], stream)
+                                      self.info[4:5], stream)
         mark("quant")
         return QuantResult(self.codes, self.scales, self.zeros, self.W_rot,
                            self.s_x, self.s_g, self.sens)
@@ -108,9 +111,9 @@ class SublayerEngine:
     def check_info(self):
         """Raises KronqError for a non-zero device status word (syncs)."""
         vals = self.info.tolist()
-        names = (("kronq_biip", "kronq_chol_split", "kronq_quantize_split")
-                 if self.split else
-                 ("kronq_biip", "kronq_chol_inv", "kronq_quantize_sublayer"))
+        names = ("kronq_accum_cov(X)", "kronq_accum_cov(G)", "kronq_biip") + (
+            ("kronq_chol_split", "kronq_quantize_split") if self.split else
+            ("kronq_chol_inv", "kronq_quantize_sublayer"))
         for name, v in zip(names, vals):
             if v != 0:
                 raise K.KronqError(name, v & 0xFF)

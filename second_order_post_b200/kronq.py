@@ -70,7 +70,7 @@ _p, _i64, _f, _d, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
                          ctypes.c_double, ctypes.c_size_t)
 _OPTS = ctypes.POINTER(kronq_opts)
 _SIGS = {
-    "kronq_accum_cov": [_p, _p, ctypes.c_int, _i64, _i64, _i64, _f, _f, _p],
+    "kronq_accum_cov": [_p, _p, ctypes.c_int, _i64, _i64, _i64, _f, _f, _p, _p],
     "kronq_sensitivity": [_p, _p, _i64, _p, _i64, _p],
     "kronq_biip": [_p, _OPTS, _p, ctypes.c_int, _i64, _i64, _p, _p, _p, _p, _p,
                    _p, _sz, _p],
@@ -79,7 +79,8 @@ _SIGS = {
     "kronq_chol_inv": [_p, _p, _i64, _f, _p, _sz, _p],
     "kronq_quantize_sublayer": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p,
                                 _sz, _p],
-    "kronq_layer_loss": [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _sz],
+    "kronq_layer_loss": [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _sz, _p],
+    "kronq_selftest_timeout": [_p, ctypes.c_uint64, _p],
     "kronq_chol_split": [_p, _p, _i64, _f, _p, _sz, _p],
     "kronq_chol_split_point": [_i64],
     "kronq_quantize_split": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p, _sz, _p],
@@ -128,12 +129,13 @@ def _dtype(t):
 
 
 # ---------------------------------------------------------------- entry points
-def kronq_accum_cov(A, H, alpha, beta, stream=None):
-    """H = alpha * AᵀA + beta * H for A (n x d, bf16/fp32, row-major)."""
+def kronq_accum_cov(A, H, alpha, beta, info, stream=None):
+    """H = alpha * AᵀA + beta * H for A (n x d, bf16/fp32, row-major); info is
+    a device int32 word (TIMEOUT when a pipeline wait ran out)."""
     n, d = A.shape
     _check("kronq_accum_cov", _lib.kronq_accum_cov(
         _stream(stream), _ptr(A), _dtype(A), n, d, A.stride(0), alpha, beta,
-        _ptr(H)))
+        _ptr(H), _ptr(info)))
 
 
 def kronq_sensitivity(H_X, H_G, out, stream=None):
@@ -200,11 +202,18 @@ def kronq_quantize_split(opts, W_rot, F, codes, scales, zeros, ws, info,
         ws.numel() * ws.element_size(), _ptr(info)))
 
 
-def kronq_layer_loss(W_ref, W_hat, H_X, H_G, loss, ws, stream=None):
+def kronq_layer_loss(W_ref, W_hat, H_X, H_G, loss, ws, info, stream=None):
     d_out, d_in = W_ref.shape
     _check("kronq_layer_loss", _lib.kronq_layer_loss(
         _stream(stream), _ptr(W_ref), _ptr(W_hat), _ptr(H_X), _ptr(H_G), d_out,
-        d_in, _ptr(loss), _ptr(ws), ws.numel() * ws.element_size()))
+        d_in, _ptr(loss), _ptr(ws), ws.numel() * ws.element_size(), _ptr(info)))
+
+
+def kronq_selftest_timeout(limit_ns, info, stream=None):
+    """Runs the library's bounded device wait on a barrier nothing completes;
+    *info becomes KRONQ_ERR_TIMEOUT after about limit_ns (<= 1e9)."""
+    _check("kronq_selftest_timeout", _lib.kronq_selftest_timeout(
+        _stream(stream), int(limit_ns), _ptr(info)))
 
 
 def kronq_gemm_f32(A, B, C, info, alpha=1.0, beta=0.0, a_mn=False, b_mn=False,

@@ -56,9 +56,14 @@ def test_last_cuda_error_and_error_text(K):
 def test_invalid_args_rejected_before_device(K):
     lib = K._lib
     nullp = ctypes.c_void_p(0)
-    assert lib.kronq_accum_cov(None, nullp, 0, 8, 8, 8, 1.0, 0.0, nullp) == K.KRONQ_ERR_INVALID_ARG
-    assert lib.kronq_accum_cov(None, ctypes.c_void_p(16), 7, 8, 8, 8, 1.0, 0.0,
-                               ctypes.c_void_p(16)) == K.KRONQ_ERR_INVALID_ARG
+    p16 = ctypes.c_void_p(16)
+    assert lib.kronq_accum_cov(None, nullp, 0, 8, 8, 8, 1.0, 0.0, nullp, p16) == K.KRONQ_ERR_INVALID_ARG
+    assert lib.kronq_accum_cov(None, p16, 7, 8, 8, 8, 1.0, 0.0, p16, p16) == K.KRONQ_ERR_INVALID_ARG
+    # the status word is required
+    assert lib.kronq_accum_cov(None, p16, 0, 8, 8, 8, 1.0, 0.0, p16, nullp) == K.KRONQ_ERR_INVALID_ARG
+    assert lib.kronq_selftest_timeout(None, 0, p16) == K.KRONQ_ERR_INVALID_ARG
+    assert lib.kronq_selftest_timeout(None, 2 * 10 ** 9, p16) == K.KRONQ_ERR_INVALID_ARG
+    assert lib.kronq_selftest_timeout(None, 1000, nullp) == K.KRONQ_ERR_INVALID_ARG
     assert lib.kronq_sensitivity(None, nullp, 4, nullp, 4, nullp) == K.KRONQ_ERR_INVALID_ARG
     o = K.make_opts(bits=5, rot_in=(256, 1), rot_out=(256, 1))
     p = ctypes.c_void_p(256)

@@ -55,8 +55,10 @@ def dev(x, dtype=None):
 def test_cov_bf16(cuda_device, n, d):
     X = synth.make_activations(n, d, -1, 1, torch.bfloat16, seed=n + d)
     H = torch.empty(d, d, device="cuda")
-    K().kronq_accum_cov(X.cuda(), H, 1.0 / n, 0.0)
+    info = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    K().kronq_accum_cov(X.cuda(), H, 1.0 / n, 0.0, info)
     torch.cuda.synchronize()
+    assert info.item() == 0
     want = O.cov(X.float().numpy())
     got = f64(H)
     assert rel_fro(got, want) < 1e-4
@@ -69,8 +71,9 @@ def test_cov_bf16_accumulates_with_beta(cuda_device):
     X1 = synth.make_activations(n, d, -1, 1, torch.bfloat16, seed=1)
     X2 = synth.make_activations(n, d, -1, 1, torch.bfloat16, seed=2)
     H = torch.empty(d, d, device="cuda")
-    K().kronq_accum_cov(X1.cuda(), H, 1.0 / n, 0.0)
-    K().kronq_accum_cov(X2.cuda(), H, 0.5 / n, 0.5)      # mean of two batches
+    info = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K().kronq_accum_cov(X1.cuda(), H, 1.0 / n, 0.0, info)
+    K().kronq_accum_cov(X2.cuda(), H, 0.5 / n, 0.5, info)      # mean of two batches
     torch.cuda.synchronize()
     want = O.cov(torch.cat([X1, X2]).float().numpy())
     assert rel_fro(f64(H), want) < 1e-4
@@ -80,8 +83,10 @@ def test_cov_bf16_accumulates_with_beta(cuda_device):
 def test_cov_f32(cuda_device, n, d):
     X = synth.make_activations(n, d, -1, 1, torch.float32, seed=7)
     H = torch.empty(d, d, device="cuda")
-    K().kronq_accum_cov(X.cuda(), H, 1.0 / n, 0.0)
+    info = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    K().kronq_accum_cov(X.cuda(), H, 1.0 / n, 0.0, info)
     torch.cuda.synchronize()
+    assert info.item() == 0
     assert rel_fro(f64(H), O.cov(X.numpy())) < 1e-5
     assert torch.equal(H, H.T)
 
@@ -383,8 +388,10 @@ def test_layer_loss(cuda_device, d_out, d_in):
     loss = torch.zeros(1, dtype=torch.float64, device="cuda")
     ws = torch.empty(Kq.kronq_workspace_bytes(Kq.KRONQ_WS_LOSS, d_out, d_in),
                      dtype=torch.uint8, device="cuda")
-    Kq.kronq_layer_loss(dev(a), dev(b), hx.cuda(), hg.cuda(), loss, ws)
+    info = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    Kq.kronq_layer_loss(dev(a), dev(b), hx.cuda(), hg.cuda(), loss, ws, info)
     torch.cuda.synchronize()
+    assert info.item() == 0
     want = O.layer_loss(a.astype(np.float64) - b, hx.double().numpy(), hg.double().numpy())
     # error budget of the two fp32-accurate products P = D H_X, Q = H_G D
     # (per element as in test_gemm_f32) carried through sum(P * Q)

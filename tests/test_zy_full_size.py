@@ -60,21 +60,21 @@ def run(cuda_device):
     eng = SublayerEngine(wl.d_out, wl.d_in, bits=wl.bits, group=wl.group,
                          damp_rel=wl.damp_rel, rot_in=wl.rot_in, rot_out=wl.rot_out)
     n = X.shape[0]
-    K.kronq_accum_cov(X, eng.H_X, 1.0 / n, 0.0)
-    K.kronq_accum_cov(G, eng.H_G, 1.0 / n, 0.0)
+    K.kronq_accum_cov(X, eng.H_X, 1.0 / n, 0.0, eng.info[0:1])
+    K.kronq_accum_cov(G, eng.H_G, 1.0 / n, 0.0, eng.info[1:2])
     K.kronq_sensitivity(eng.H_X, eng.H_G, eng.sens)
     HX0, HG0 = eng.H_X.clone(), eng.H_G.clone()
     K.kronq_biip(eng.opts, W, eng.W_rot, eng.H_X, eng.H_G, eng.s_x, eng.s_g,
-                 eng.ws, eng.info[0:1])
+                 eng.ws, eng.info[2:3])
     HX1, W1 = eng.H_X.clone(), eng.W_rot.clone()
     if eng.split:   # the engine's choice for this shape (d_in > d_out)
-        K.kronq_chol_split(eng.H_X, wl.damp_rel, eng.ws, eng.info[1:2])
+        K.kronq_chol_split(eng.H_X, wl.damp_rel, eng.ws, eng.info[3:4])
         K.kronq_quantize_split(eng.opts, eng.W_rot, eng.H_X, eng.codes, eng.scales,
-                               eng.zeros, eng.ws, eng.info[2:3])
+                               eng.zeros, eng.ws, eng.info[4:5])
     else:
-        K.kronq_chol_inv(eng.H_X, wl.damp_rel, eng.ws, eng.info[1:2])
+        K.kronq_chol_inv(eng.H_X, wl.damp_rel, eng.ws, eng.info[3:4])
         K.kronq_quantize_sublayer(eng.opts, eng.W_rot, eng.H_X, eng.codes, eng.scales,
-                                  eng.zeros, eng.ws, eng.info[2:3])
+                                  eng.zeros, eng.ws, eng.info[4:5])
     torch.cuda.synchronize()
     eng.check_info()
     return dict(wl=wl, W=W, X=X, G=G, eng=eng, HX0=HX0, HG0=HG0, HX1=HX1, W1=W1)
