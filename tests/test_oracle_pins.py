@@ -48,6 +48,53 @@ def test_gaussian_draws_are_standard_normal():
     assert scipy.stats.kstest(g, "norm").pvalue > 1e-3
 
 
+def _rotation_golden():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "rotation_seed0.txt"))
+            if l.strip() and not l.startswith("#")]
+    return rows
+
+
+def test_side_keys_draws_and_signs_seed0():
+    # hand-worked values of key = sm64(sm64(seed) + side) and the sign rule
+    for row in _rotation_golden():
+        kind, side = row[0], int(row[1])
+        key = O.side_key(0, side)
+        if kind == "key":
+            assert int(key) == int(row[2], 16)
+        elif kind == "draws":
+            got = O.sm64(np.uint64(key) + np.arange(8, dtype=np.uint64))
+            assert [int(x) for x in got] == [int(v, 16) for v in row[2:]]
+        elif kind == "signs":
+            want = [1.0 if c == "+" else -1.0 for c in row[2:]]
+            assert O.rotation_signs(0, side, 8).tolist() == want
+        elif kind == "kq":
+            assert int(key ^ np.uint64(0xA5A5A5A5A5A5A5A5)) == int(row[2], 16)
+
+
+def test_first_box_muller_normals_seed0():
+    # G[0][0] and G[0][1] of each side (counter t = 0, 1), hand-worked
+    for row in _rotation_golden():
+        if row[0] != "normal":
+            continue
+        side, t = int(row[1]), int(row[2])
+        g = O.gaussian_matrix(0, side, 2)
+        assert math.isclose(g[0, t], float(row[7]), rel_tol=1e-13)
+
+
+def test_diag_scale_hand_examples():
+    # floor = 1e-8 * mean of the diagonal as given, then the power
+    for line in open(os.path.join(GOLDEN, "diag_scale_examples.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        e, dg, want = (part.split() for part in line.split("|"))
+        e = float(e[0])
+        dg = np.array([float(x) for x in dg])
+        want = np.array([eval(x, {"__builtins__": {}}) for x in want])
+        got = O.diag_scale_of(dg, e)
+        assert np.allclose(got, want, rtol=1e-13, atol=0)
+        assert np.allclose(O.diag_scale(np.diag(dg), e), want, rtol=1e-13, atol=0)
+
+
 @pytest.mark.parametrize("m", [1, 2, 28, 172])
 def test_q_factor_is_the_qr_orthogonal_factor(m):
     q = O.q_factor(3, 1, m)
