@@ -532,6 +532,580 @@ __global__ void __launch_bounds__(512)
   }
 }
 
+// ------------------------------------------------------------- column pass
+// The whole row side of a rotation in one read and one write of the matrix:
+// for every column x of an R x C row-major matrix (R = had * m),
+//   x <- (Hhat_had ⊗ Q_m) x      (Hadamard unnormalised; the row pass has
+//                                 applied the row factors and the norm)
+// in place. A strip of 4*W4 contiguous columns is held, over all R rows, in
+// the shared memory of a cluster of K CTAs: CTA k holds rows
+// [k*RK, (k+1)*RK), RK = (had/K)*m, i.e. Hadamard index a in
+// [k*had/K, (k+1)*had/K). Each CTA mixes its groups of m rows with Q_m and
+// runs the Hadamard over its local low bits of a; after a cluster barrier the
+// high log2(K) bits are one K-point Hadamard across the CTAs, read through
+// distributed shared memory, and each CTA writes its share of the positions
+// for all K row blocks straight to global memory.
+constexpr int CP_THREADS = 256;
+constexpr int CP_BUDGET = 112 * 1024;   // dynamic shared memory per CTA (2 per SM)
+
+struct ColP {
+  float *M;
+  int64_t ld, C;
+  int had, m, W4;   // W4: float4 columns per strip
+  int box;          // rows per TMA box (divides the rows a CTA holds)
+  const float *Q;   // m x m row-major (m > 1, m % 4 == 0), else null
+  int32_t *info;
+};
+
+// y = Q x for each group of m rows, one thread per (group, column pair); x is
+// held in registers, Q rows are read as float4 broadcasts through L1.
+__device__ void colpass_qmix(float *X, int AL, int m, int W4, const float *Q) {
+  const int W2 = 2 * W4, W = 4 * W4;
+  const float4 *Q4 = reinterpret_cast<const float4 *>(Q);
+  const int m4 = m / 4;
+  for (int t = threadIdx.x; t < AL * W2; t += CP_THREADS) {
+    const int al = t / W2, c2 = t % W2;
+    float2 *base = reinterpret_cast<float2 *>(X + static_cast<int64_t>(al) * m * W) + c2;
+    float2 x[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) x[k] = k < m ? base[k * W2] : make_float2(0.f, 0.f);
+    for (int b = 0; b < m; ++b) {
+      const float4 *qr = Q4 + b * m4;
+      float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        if (k4 < m4) {
+          const float4 q = __ldg(qr + k4);
+          y.x = fmaf(q.x, x[4 * k4].x, y.x);
+          y.y = fmaf(q.x, x[4 * k4].y, y.y);
+          y.x = fmaf(q.y, x[4 * k4 + 1].x, y.x);
+          y.y = fmaf(q.y, x[4 * k4 + 1].y, y.y);
+          y.x = fmaf(q.z, x[4 * k4 + 2].x, y.x);
+          y.y = fmaf(q.z, x[4 * k4 + 2].y, y.y);
+          y.x = fmaf(q.w, x[4 * k4 + 3].x, y.x);
+          y.y = fmaf(q.w, x[4 * k4 + 3].y, y.y);
+        }
+      }
+      base[b * W2] = y;
+    }
+  }
+  __syncthreads();
+}
+
+template <int K>
+__global__ void __launch_bounds__(CP_THREADS, 2)
+    colpass_kernel(const __grid_constant__ CUtensorMap tm, ColP p) {
+  extern __shared__ __align__(128) float4 X4[];
+  const int rank = K > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int64_t strip = blockIdx.x / K;
+  const int m = p.m, W4 = p.W4;
+  const int AL = p.had / K, RK = AL * m;
+  const int nvec = RK * W4;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(X4 + nvec);
+  int *abort_flag = reinterpret_cast<int *>(bar + 1);
+  const int64_t row0 = static_cast<int64_t>(rank) * RK;
+  const int64_t c0 = strip * 4 * W4;
+  // 1. the CTA's row block of the strip, by TMA (columns beyond C read as 0)
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm);
+    mbar_expect_tx(bar, static_cast<uint32_t>(nvec) * 16u);
+    for (int r = 0; r < RK; r += p.box)
+      tma_load_2d(X4 + r * W4, &tm, bar, static_cast<int32_t>(c0),
+                  static_cast<int32_t>(row0 + r));
+  }
+  __syncthreads();
+  const bool landed = mbar_wait(bar, 0, abort_flag);
+  const int good = __syncthreads_and(landed);
+  if (!good && threadIdx.x == 0) report(p.info, KRONQ_ERR_TIMEOUT);
+  if (good) {
+    // 2. Q_m over each group of m consecutive rows
+    if (m > 1) colpass_qmix(reinterpret_cast<float *>(X4), AL, m, W4, p.Q);
+    // 3. Hadamard over the local bits of a (rows al*m + b, stride m rows)
+    if (AL > 1) {
+      int h = 1;
+      while (AL / h >= 16) {
+        round4_smem<16>(X4, AL, h, m * W4);
+        h *= 16;
+      }
+      switch (AL / h) {
+        case 8: round4_smem<8>(X4, AL, h, m * W4); break;
+        case 4: round4_smem<4>(X4, AL, h, m * W4); break;
+        case 2: round4_smem<2>(X4, AL, h, m * W4); break;
+        default: break;
+      }
+    }
+  }
+  // 4. the high bits of a: a K-point Hadamard across the cluster (every CTA
+  // takes the same barriers, also after a timeout)
+  if (K > 1) cluster_sync_all();
+  if (good) {
+    const int per = (nvec + K - 1) / K;
+    const int p0 = rank * per, p1 = min(nvec, p0 + per);
+    const uint32_t xs = smem_u32(X4);
+    for (int q = p0 + threadIdx.x; q < p1; q += CP_THREADS) {
+      float4 v[K];
+#pragma unroll
+      for (int j = 0; j < K; ++j)
+        v[j] = (K == 1 || j == rank) ? X4[q]
+                                     : ld_dsmem_f4(mapa_shared(xs + 16u * q, j));
+      fwht_reg4<K>(v);
+      const int r = q / W4, c4 = q % W4;
+      const int64_t col = c0 + 4 * c4;
+      if (col < p.C) {
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+          __stcs(reinterpret_cast<float4 *>(p.M + (static_cast<int64_t>(j) * RK + r) * p.ld + col),
+                 v[j]);
+      }
+    }
+  }
+  // no CTA leaves while another may still read its shared memory
+  if (K > 1) cluster_sync_all();
+  if (!good && threadIdx.x == 0) {
+    // let a late copy land before the shared memory is released
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, 0) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+}
+
+template <int K, int M, int AL>
+__global__ void __launch_bounds__(CP_THREADS, 2)
+    colpass_tpl_kernel(const __grid_constant__ CUtensorMap tm, ColP p);
+
+// Plans and launches the column pass; returns KRONQ_ERR_UNSUPPORTED when the
+// shape does not fit it (the caller then takes the two-pass route).
+kronq_status launch_colpass(cudaStream_t st, float *M, int64_t ld, int64_t R,
+                            int64_t C, int64_t had, int64_t m, const float *Q,
+                            int32_t *info) {
+  if (m > 32 || (m > 1 && (m % 4 != 0 || Q == nullptr)) || had < 1 || had * m != R)
+    return KRONQ_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(M) % 16 || ld % 4 || C % 4)
+    return KRONQ_ERR_UNSUPPORTED;
+  int W4 = 0, K = 0;
+  for (int w4 : {4, 2, 1}) {
+    int k = 1;
+    while (static_cast<int64_t>(k) * CP_BUDGET < R * w4 * 16) k *= 2;
+    if (k <= 16 && k <= had) {
+      W4 = w4;
+      K = k;
+      break;
+    }
+  }
+  if (K == 0) return KRONQ_ERR_UNSUPPORTED;
+  const int64_t strips = ceil_div(C, 4 * W4);
+  if (strips * K > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+  const int64_t AL = had / K, RK = AL * m;
+  // rows per TMA box: a divisor of RK of at most 256
+  int64_t box = 1;
+  if (RK <= 256) {
+    box = RK;
+  } else if (RK % 256 == 0) {
+    box = 256;
+  } else {
+    for (int64_t dv = 1; dv <= m; ++dv)
+      if (m % dv == 0 && AL * dv <= 256) box = kq_max(box, AL * dv);
+  }
+  CUtensorMap tm;
+  KQ_TRY(make_tmap_2d(&tm, M, false, static_cast<uint64_t>(C), static_cast<uint64_t>(R),
+                      static_cast<uint64_t>(ld), static_cast<uint32_t>(4 * W4),
+                      static_cast<uint32_t>(box), TMAP_NONE));
+  const int smem = static_cast<int>(RK * W4 * 16 + 64);
+  ColP p{M, ld, C, static_cast<int>(had), static_cast<int>(m), W4, static_cast<int>(box), Q,
+         info};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(strips * K));
+  cfg.blockDim = dim3(CP_THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(K);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = K > 1 ? 1 : 0;
+  auto go = [&](auto kern) -> kronq_status {
+    KQ_TRY(smem_attr(kern, CP_BUDGET + 64));
+    if (K > 8) KQ_TRY(nonportable_cluster_attr(kern));
+    KQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tm, p));
+    count_launch();
+    return KRONQ_OK;
+  };
+  if (W4 == 4) {  // the compiled fixed shapes
+#define KQ_COL_SHAPE(KK, MM, AA)                                              \
+  if (K == KK && m == MM && AL == AA) return go(colpass_tpl_kernel<KK, MM, AA>);
+    KQ_COL_SHAPE(16, 28, 64)
+    KQ_COL_SHAPE(16, 1, 1024)
+    KQ_COL_SHAPE(8, 1, 1024)
+    KQ_COL_SHAPE(4, 1, 1024)
+    KQ_COL_SHAPE(2, 1, 1024)
+    KQ_COL_SHAPE(1, 1, 1024)
+    KQ_COL_SHAPE(1, 1, 512)
+    KQ_COL_SHAPE(1, 1, 256)
+#undef KQ_COL_SHAPE
+  }
+  switch (K) {
+    case 1: return go(colpass_kernel<1>);
+    case 2: return go(colpass_kernel<2>);
+    case 4: return go(colpass_kernel<4>);
+    case 8: return go(colpass_kernel<8>);
+    default: return go(colpass_kernel<16>);
+  }
+}
+
+// ------------------------------------------------------------- fixed shapes
+// The shapes of the pages' sublayers (row chunks of L*M floats with M = 1 or
+// 28; column strips over R = had*M rows) with every size a compile-time
+// constant: the index arithmetic of the inner loops is shifts and multiplies,
+// and the Hadamard runs in rounds of radix 32.
+
+// Radix of the next round when n Hadamard points remain (at most rmax):
+// everything at once when n <= rmax, else balanced rounds.
+__host__ __device__ constexpr int radix_for(int n, int rmax) {
+  if (n <= rmax) return n;
+  if (n > rmax * rmax) return rmax;
+  int r = 1;
+  while (r * r < n) r *= 2;
+  return r;
+}
+
+template <int L, int H>
+struct RadixAt {
+  static constexpr int R = radix_for(L / H, 32);
+};
+
+// distance of the last round of that plan, from distance 1 upward
+__host__ __device__ constexpr int last_round_h(int L) {
+  int h = 1;
+  while (true) {
+    const int r = radix_for(L / h, 32);
+    if (h * r >= L) return h;
+    h *= r;
+  }
+}
+
+// One round of radix R at distance H over the a-index of an L x M chunk in
+// shared memory (element a*M + b), tasks (g, b).
+template <int L, int M, int R, int H, int NT>
+__device__ __forceinline__ void tround(float *X) {
+  constexpr int T = (L / R) * M;
+  for (int t = threadIdx.x; t < T; t += NT) {
+    const int b = t % M, g = t / M;
+    const int a = (g / H) * R * H + (g % H);
+    float *x = X + a * M + b;
+    float r[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) r[i] = x[i * H * M];
+    fwht_reg<R>(r);
+#pragma unroll
+    for (int i = 0; i < R; ++i) x[i * H * M] = r[i];
+  }
+  __syncthreads();
+}
+
+// Rounds from distance H up to (but not including) distance HEND.
+template <int L, int M, int H, int HEND, int NT>
+__device__ __forceinline__ void trounds(float *X) {
+  if constexpr (H < HEND) {
+    constexpr int R = RadixAt<L, H>::R;
+    tround<L, M, R, H, NT>(X);
+    trounds<L, M, H * R, HEND, NT>(X);
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float4 load4(const void *base, int64_t off) {
+  if constexpr (BF16) {
+    const uint2 u = __ldcs(reinterpret_cast<const uint2 *>(
+        reinterpret_cast<const __nv_bfloat16 *>(base) + off));
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+    return make_float4(a.x, a.y, b.x, b.y);
+  } else {
+    return __ldcs(reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + off));
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float load1(const void *base, int64_t off) {
+  if constexpr (BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[off]);
+  else return __ldcs(reinterpret_cast<const float *>(base) + off);
+}
+
+constexpr int RT_THREADS = 512;
+
+// Row pass, one CTA per row chunk of L*M contiguous columns:
+// out = norm * cr[row] * (Hhat_L ⊗ Q_M)(cc ⊙ x) (unnormalised Hadamard times
+// norm). M == 1: vector loads into shared memory, the last Hadamard round
+// fused with the store. M > 1: the first round (radix 16) fused with the
+// loads, the Q_M mix with the store (lane b holds row b of Q_M).
+template <int L, int M, bool BF16>
+__global__ void __launch_bounds__(RT_THREADS, 2) row_tpl_kernel(RowP p) {
+  extern __shared__ float X[];
+  constexpr int CH = L * M;
+  const int64_t row = blockIdx.x / p.chunks;
+  const int64_t c0 = (blockIdx.x % p.chunks) * CH;
+  const float rf = p.norm * (p.cr ? p.cr[row] : 1.f);
+  const float *cc = p.cc ? p.cc + c0 : nullptr;
+  const int64_t in0 = row * p.ld_in + c0;
+  float *o = p.out + row * p.ld_out + c0;
+  if constexpr (M == 1) {
+    float4 *X4 = reinterpret_cast<float4 *>(X);
+    for (int e4 = threadIdx.x; e4 < CH / 4; e4 += RT_THREADS) {
+      float4 v = load4<BF16>(p.in, in0 + 4 * e4);
+      float4 f = make_float4(rf, rf, rf, rf);
+      if (cc) {
+        const float4 c = __ldg(reinterpret_cast<const float4 *>(cc) + e4);
+        f = make_float4(rf * c.x, rf * c.y, rf * c.z, rf * c.w);
+      }
+      X4[e4] = make_float4(v.x * f.x, v.y * f.y, v.z * f.z, v.w * f.w);
+    }
+    __syncthreads();
+    constexpr int HL = last_round_h(L);
+    constexpr int RL = L / HL;
+    trounds<L, 1, 1, HL, RT_THREADS>(X);
+    for (int t = threadIdx.x; t < L / RL; t += RT_THREADS) {
+      const int a = (t / HL) * RL * HL + (t % HL);
+      float r[RL];
+#pragma unroll
+      for (int i = 0; i < RL; ++i) r[i] = X[a + i * HL];
+      fwht_reg<RL>(r);
+#pragma unroll
+      for (int i = 0; i < RL; ++i) o[a + i * HL] = r[i];
+    }
+  } else {
+    constexpr int R0 = L >= 32 ? 32 : L;
+    for (int t = threadIdx.x; t < (L / R0) * M; t += RT_THREADS) {
+      const int b = t % M, g = t / M;
+      const int e0 = g * R0 * M + b;
+      float r[R0];
+#pragma unroll
+      for (int i = 0; i < R0; ++i) {
+        const int e = e0 + i * M;
+        float v = load1<BF16>(p.in, in0 + e) * rf;
+        if (cc) v *= __ldg(cc + e);
+        r[i] = v;
+      }
+      fwht_reg<R0>(r);
+#pragma unroll
+      for (int i = 0; i < R0; ++i) X[e0 + i * M] = r[i];
+    }
+    __syncthreads();
+    trounds<L, M, R0, L, RT_THREADS>(X);
+    // Q_M mix on the way out, two groups per warp iteration
+    static_assert(M % 4 == 0 && M <= 32, "Q_M mix needs M % 4 == 0, M <= 32");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = RT_THREADS / 32;
+    float q[M];
+#pragma unroll
+    for (int k = 0; k < M; ++k) q[k] = lane < M ? __ldg(p.Q + lane * M + k) : 0.f;
+    static_assert(L % 4 == 0, "four groups per warp iteration");
+    for (int a = 4 * warp; a < L; a += 4 * NW) {
+      const float4 *x0 = reinterpret_cast<const float4 *>(X + a * M);
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k4 = 0; k4 < M / 4; ++k4) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 u = x0[g * (M / 4) + k4];
+          y[g] = fmaf(q[4 * k4], u.x, y[g]);
+          y[g] = fmaf(q[4 * k4 + 1], u.y, y[g]);
+          y[g] = fmaf(q[4 * k4 + 2], u.z, y[g]);
+          y[g] = fmaf(q[4 * k4 + 3], u.w, y[g]);
+        }
+      }
+      if (lane < M) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) o[(a + g) * M + lane] = y[g];
+      }
+    }
+  }
+}
+
+// Launches the fixed-shape row pass when (L, M, dtype) is one of the
+// compiled shapes; KRONQ_ERR_UNSUPPORTED otherwise.
+kronq_status launch_row_tpl(cudaStream_t st, const RowP &p, int64_t rows, bool bf16) {
+  const int L = p.L, M = p.m;
+  if (reinterpret_cast<uintptr_t>(p.out) % 16 || p.ld_out % 4 || p.ld_in % 4 ||
+      reinterpret_cast<uintptr_t>(p.in) % 16 || (p.cc && reinterpret_cast<uintptr_t>(p.cc) % 16) ||
+      (M > 1 && p.Q == nullptr))
+    return KRONQ_ERR_UNSUPPORTED;
+  const int64_t blocks = rows * p.chunks;
+  if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+  const int smem = L * M * 4;
+  auto go = [&](auto kern) -> kronq_status {
+    KQ_TRY(smem_attr(kern, smem));
+    kern<<<static_cast<unsigned>(blocks), RT_THREADS, smem, st>>>(p);
+    KQ_CHECK_LAUNCH();
+    return KRONQ_OK;
+  };
+#define KQ_ROW_SHAPE(LL, MM)                                                  \
+  if (L == LL && M == MM)                                                     \
+    return bf16 ? go(row_tpl_kernel<LL, MM, true>) : go(row_tpl_kernel<LL, MM, false>);
+  KQ_ROW_SHAPE(256, 1)
+  KQ_ROW_SHAPE(512, 1)
+  KQ_ROW_SHAPE(1024, 1)
+  KQ_ROW_SHAPE(2048, 1)
+  KQ_ROW_SHAPE(4096, 1)
+  KQ_ROW_SHAPE(8192, 1)
+  KQ_ROW_SHAPE(16384, 1)
+  KQ_ROW_SHAPE(256, 28)
+  KQ_ROW_SHAPE(512, 28)
+  KQ_ROW_SHAPE(1024, 28)
+#undef KQ_ROW_SHAPE
+  return KRONQ_ERR_UNSUPPORTED;
+}
+
+// rows per TMA box for the column pass: a divisor of RK = AL * M of at most 256
+__host__ __device__ constexpr int colpass_box(int AL, int M) {
+  const int RK = AL * M;
+  if (RK <= 256) return RK;
+  if (RK % 256 == 0) return 256;
+  int best = 1;
+  for (int dv = 1; dv <= M; ++dv)
+    if (M % dv == 0 && AL * dv <= 256 && AL * dv > best) best = AL * dv;
+  return best;
+}
+
+// One Hadamard round over the local a-index of a column strip held as float4
+// vectors (V = M * 4 vectors per a).
+template <int AL, int V, int R, int H>
+__device__ __forceinline__ void tround4(float4 *X4) {
+  constexpr int T = (AL / R) * V;
+  for (int t = threadIdx.x; t < T; t += CP_THREADS) {
+    const int v = t % V, g = t / V;
+    const int a = (g / H) * R * H + (g % H);
+    float4 *x = X4 + a * V + v;
+    float4 r[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) r[i] = x[i * H * V];
+    fwht_reg4<R>(r);
+#pragma unroll
+    for (int i = 0; i < R; ++i) x[i * H * V] = r[i];
+  }
+  __syncthreads();
+}
+
+template <int AL, int V, int H>
+__device__ __forceinline__ void trounds4(float4 *X4) {
+  if constexpr (H < AL) {
+    constexpr int R = radix_for(AL / H, 16);
+    tround4<AL, V, R, H>(X4);
+    trounds4<AL, V, H * R>(X4);
+  }
+}
+
+// Column pass (see colpass_kernel) with K, M and the local Hadamard length AL
+// fixed at compile time and strips of 16 columns.
+template <int K, int M, int AL>
+__global__ void __launch_bounds__(CP_THREADS, 2)
+    colpass_tpl_kernel(const __grid_constant__ CUtensorMap tm, ColP p) {
+  extern __shared__ __align__(128) float4 X4[];
+  constexpr int W4 = 4, RK = AL * M, NV = RK * W4, BOX = colpass_box(AL, M);
+  const int rank = K > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int64_t strip = blockIdx.x / K;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(X4 + NV);
+  int *abort_flag = reinterpret_cast<int *>(bar + 1);
+  const int64_t row0 = static_cast<int64_t>(rank) * RK;
+  const int64_t c0 = strip * 4 * W4;
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm);
+    mbar_expect_tx(bar, static_cast<uint32_t>(NV) * 16u);
+#pragma unroll 1
+    for (int r = 0; r < RK; r += BOX)
+      tma_load_2d(X4 + r * W4, &tm, bar, static_cast<int32_t>(c0),
+                  static_cast<int32_t>(row0 + r));
+  }
+  __syncthreads();
+  const bool landed = mbar_wait(bar, 0, abort_flag);
+  const int good = __syncthreads_and(landed);
+  if (!good && threadIdx.x == 0) report(p.info, KRONQ_ERR_TIMEOUT);
+  if (good) {
+    if constexpr (M > 1) {
+      // Q_M over each group of M rows: one thread per (group, column pair)
+      constexpr int W2 = 2 * W4, W = 4 * W4, M4 = M / 4;
+      static_assert(M % 4 == 0, "Q_M mix needs M % 4 == 0");
+      float *X = reinterpret_cast<float *>(X4);
+      const float4 *Q4 = reinterpret_cast<const float4 *>(p.Q);
+      for (int t = threadIdx.x; t < AL * W2; t += CP_THREADS) {
+        const int al = t / W2, c2 = t % W2;
+        float2 *base = reinterpret_cast<float2 *>(X + al * M * W) + c2;
+        float2 x[M];
+#pragma unroll
+        for (int k = 0; k < M; ++k) x[k] = base[k * W2];
+        // two output rows per step: four independent FMA chains
+#pragma unroll
+        for (int b = 0; b < M; b += 2) {
+          const float4 *q0r = Q4 + b * M4, *q1r = q0r + M4;
+          float2 y0 = make_float2(0.f, 0.f), y1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int k4 = 0; k4 < M4; ++k4) {
+            const float4 q0 = __ldg(q0r + k4), q1 = __ldg(q1r + k4);
+            const float2 u0 = x[4 * k4], u1 = x[4 * k4 + 1];
+            const float2 u2 = x[4 * k4 + 2], u3 = x[4 * k4 + 3];
+            y0.x = fmaf(q0.x, u0.x, y0.x);
+            y0.y = fmaf(q0.x, u0.y, y0.y);
+            y1.x = fmaf(q1.x, u0.x, y1.x);
+            y1.y = fmaf(q1.x, u0.y, y1.y);
+            y0.x = fmaf(q0.y, u1.x, y0.x);
+            y0.y = fmaf(q0.y, u1.y, y0.y);
+            y1.x = fmaf(q1.y, u1.x, y1.x);
+            y1.y = fmaf(q1.y, u1.y, y1.y);
+            y0.x = fmaf(q0.z, u2.x, y0.x);
+            y0.y = fmaf(q0.z, u2.y, y0.y);
+            y1.x = fmaf(q1.z, u2.x, y1.x);
+            y1.y = fmaf(q1.z, u2.y, y1.y);
+            y0.x = fmaf(q0.w, u3.x, y0.x);
+            y0.y = fmaf(q0.w, u3.y, y0.y);
+            y1.x = fmaf(q1.w, u3.x, y1.x);
+            y1.y = fmaf(q1.w, u3.y, y1.y);
+          }
+          base[b * W2] = y0;
+          base[(b + 1) * W2] = y1;
+        }
+      }
+      __syncthreads();
+    }
+    trounds4<AL, M * W4, 1>(X4);
+  }
+  if (K > 1) cluster_sync_all();
+  if (good) {
+    constexpr int PER = (NV + K - 1) / K;
+    const int p0 = rank * PER, p1 = min(NV, p0 + PER);
+    const uint32_t xs = smem_u32(X4);
+    for (int q = p0 + threadIdx.x; q < p1; q += CP_THREADS) {
+      float4 v[K];
+#pragma unroll
+      for (int j = 0; j < K; ++j)
+        v[j] = (K == 1 || j == rank) ? X4[q]
+                                     : ld_dsmem_f4(mapa_shared(xs + 16u * q, j));
+      fwht_reg4<K>(v);
+      const int r = q / W4, c4 = q % W4;
+      const int64_t col = c0 + 4 * c4;
+      if (col < p.C) {
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+          __stcs(reinterpret_cast<float4 *>(p.M + (static_cast<int64_t>(j) * RK + r) * p.ld + col),
+                 v[j]);
+      }
+    }
+  }
+  if (K > 1) cluster_sync_all();
+  if (!good && threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, 0) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+}
+
 // ------------------------------------------------------------- planning
 struct SideRot {
   int64_t d, had, m;
@@ -588,7 +1162,7 @@ kronq_status launch_strided(cudaStream_t st, float *base, int64_t outer,
 kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in,
                     float *out, int64_t ld_out, int64_t R, int64_t C,
                     const SideRot &sr, const SideRot &sc, const float *cr,
-                    const float *cc) {
+                    const float *cc, int32_t *info) {
   const int64_t had_r = sr.rot ? sr.had : 1, m_r = sr.rot ? sr.m : 1;
   const int64_t had_c = sc.rot ? sc.had : 1, m_c = sc.rot ? sc.m : 1;
   // ---- row pass over chunks of Lc * m_c contiguous columns
@@ -622,13 +1196,25 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
       p.m = static_cast<int>(chunk);
       p.Q = nullptr;
     }
-    row_pass_kernel<<<static_cast<unsigned>(blocks), 512, smem, st>>>(p);
-    KQ_CHECK_LAUNCH();
+    const kronq_status fast = launch_row_tpl(st, p, R, in_bf16);
+    if (fast != KRONQ_ERR_UNSUPPORTED) {
+      KQ_TRY(fast);
+    } else {
+      row_pass_kernel<<<static_cast<unsigned>(blocks), 512, smem, st>>>(p);
+      KQ_CHECK_LAUNCH();
+    }
   }
   // ---- column-side Hadamard bits beyond the chunk
   if (sc.rot && had_c / Lc > 1)
     KQ_TRY(launch_strided(st, out, R, ld_out, had_c / Lc, chunk, chunk));
-  // ---- row side: Q_m over groups of m_r consecutive rows, then the Hadamard
+  // ---- row side in one pass (cluster column pass) where the shape allows
+  if (sr.rot && (had_r > 1 || m_r > 1)) {
+    const kronq_status s = launch_colpass(st, out, ld_out, R, C, had_r, m_r,
+                                          m_r > 1 ? sr.Q : nullptr, info);
+    if (s != KRONQ_ERR_UNSUPPORTED) return s;
+  }
+  // ---- otherwise two passes: Q_m over groups of m_r consecutive rows, then
+  // the Hadamard
   if (sr.rot && m_r > 1) {
     // Q_m, then Qᵀ (m <= 32) or a [m][64] input tile (m > 32)
     const size_t smem =
@@ -693,10 +1279,10 @@ kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
   SideRot rx{d_in, o.rot_in.had, o.rot_in.m, rot_x, Qx};
   SideRot rg{d_out, o.rot_out.had, o.rot_out.m, rot_g, Qg};
   // W' = U_G (S_G W S_X) U_Xᵀ: rows use the output side, columns the input side
-  KQ_TRY(rotate(st, W, w_bf16, d_in, W_rot, d_in, d_out, d_in, rg, rx, fgw, fxw));
+  KQ_TRY(rotate(st, W, w_bf16, d_in, W_rot, d_in, d_out, d_in, rg, rx, fgw, fxw, info));
   // H_X' = U_X S_X^-1 H_X S_X^-1 U_Xᵀ, H_G' likewise (in place)
-  KQ_TRY(rotate(st, H_X, false, d_in, H_X, d_in, d_in, d_in, rx, rx, fxh, fxh));
-  KQ_TRY(rotate(st, H_G, false, d_out, H_G, d_out, d_out, d_out, rg, rg, fgh, fgh));
+  KQ_TRY(rotate(st, H_X, false, d_in, H_X, d_in, d_in, d_in, rx, rx, fxh, fxh, info));
+  KQ_TRY(rotate(st, H_G, false, d_out, H_G, d_out, d_out, d_out, rg, rg, fgh, fgh, info));
   return KRONQ_OK;
 }
 

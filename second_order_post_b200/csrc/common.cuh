@@ -54,13 +54,20 @@ template <class F>
 inline kronq_status smem_attr(F *func, int bytes) {
   return set_max_dyn_smem(reinterpret_cast<const void *>(func), bytes);
 }
+// Lets a kernel launch with clusters of more than 8 CTAs (once per device).
+kronq_status set_nonportable_cluster(const void *func);
+template <class F>
+inline kronq_status nonportable_cluster_attr(F *func) {
+  return set_nonportable_cluster(reinterpret_cast<const void *>(func));
+}
 
 // 2D tiled tensor map over a row-major fp32/bf16 matrix: inner extent `inner`
 // (contiguous), outer extent `outer`, row pitch `pitch_elems`, box
 // {box_inner, box_outer}, zero fill out of bounds. Swizzle: TMAP_SW128
 // (128-byte rows, 16-byte granules), TMAP_SW128_32B (128-byte rows, 32-byte
-// granules) or TMAP_SW64 (64-byte rows, 16-byte granules).
-enum { TMAP_SW128 = 0, TMAP_SW128_32B = 1, TMAP_SW64 = 2 };
+// granules), TMAP_SW64 (64-byte rows, 16-byte granules) or TMAP_NONE (the
+// box lands row-major and unswizzled).
+enum { TMAP_SW128 = 0, TMAP_SW128_32B = 1, TMAP_SW64 = 2, TMAP_NONE = 3 };
 kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
                           uint64_t inner, uint64_t outer, uint64_t pitch_elems,
                           uint32_t box_inner, uint32_t box_outer,
@@ -175,6 +182,16 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::"
       "bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Untiled bulk copy of `bytes` (multiple of 16; both addresses 16-byte
+// aligned) global -> shared, completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *src,
+                                          uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -307,6 +324,35 @@ __device__ __forceinline__ float tf32_lo1(float x) {
 }
 __device__ __forceinline__ float4 tf32_lo(float4 x) {
   return make_float4(tf32_lo1(x.x), tf32_lo1(x.y), tf32_lo1(x.z), tf32_lo1(x.w));
+}
+
+// ---- thread-block clusters (distributed shared memory)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster arrives (release) and waits
+// (acquire): shared-memory writes before it are visible cluster-wide after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address, in the shared::cluster window, of the same shared-memory offset in
+// the cluster's CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -107,17 +107,28 @@ kronq_status require_sm100() {
   return state == 1 ? KRONQ_OK : KRONQ_ERR_CUDA;
 }
 
-kronq_status set_max_dyn_smem(const void *func, int bytes) {
+namespace {
+// Sets a function attribute once per (device, kernel, attribute, value).
+kronq_status set_func_attr_once(const void *func, cudaFuncAttribute attr, int value) {
   int dev = -1;
   KQ_CUDA(cudaGetDevice(&dev));
   static std::mutex mu;
-  static std::set<std::tuple<int, const void *, int>> done;
+  static std::set<std::tuple<int, const void *, int, int>> done;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(dev, func, bytes);
+  const auto key = std::make_tuple(dev, func, static_cast<int>(attr), value);
   if (done.count(key)) return KRONQ_OK;
-  KQ_CUDA(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  KQ_CUDA(cudaFuncSetAttribute(func, attr, value));
   done.insert(key);
   return KRONQ_OK;
+}
+}  // namespace
+
+kronq_status set_max_dyn_smem(const void *func, int bytes) {
+  return set_func_attr_once(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+kronq_status set_nonportable_cluster(const void *func) {
+  return set_func_attr_once(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
 }
 
 kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
@@ -139,6 +150,7 @@ kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swz == TMAP_SW128_32B ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                   : swz == TMAP_SW64    ? CU_TENSOR_MAP_SWIZZLE_64B
+                  : swz == TMAP_NONE    ? CU_TENSOR_MAP_SWIZZLE_NONE
                                         : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
