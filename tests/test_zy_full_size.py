@@ -1,8 +1,14 @@
-"""Parity at the full LLaMA-3-70B down_proj size (W 8192 x 28672, 131072
-calibration tokens, W2 g128, Hadamard-1024 x Q_28 on the input side), in the
-launch configuration the benchmark times: the same C-ABI calls on the same
-buffers as SublayerEngine.run, one step at a time so that each step's input
-can be kept for the checks.
+"""Parity at the full sizes of the pages' sublayers, in the launch
+configuration the benchmark times: the same C-ABI calls on the same buffers
+as SublayerEngine.run, one step at a time so that each step's input can be
+kept for the checks. Workloads:
+  - LLaMA-3-70B down_proj: W 8192 x 28672, 131072 tokens, W2 g128,
+    Hadamard-1024 x Q_28 on the input side;
+  - LLaMA-2-7B attention: W 4096 x 4096, 262144 tokens, W2 g128;
+  - LLaMA-2-7B MLP gate/up: W 11008 x 4096, 262144 tokens, W3 g128,
+    Hadamard-64 x Q_172 on the output side;
+  - LLaMA-2-7B MLP down: W 4096 x 11008, 262144 Student-t tokens, W3 g128,
+    Hadamard-64 x Q_172 on the input side.
 
 The oracle cannot redo this size in seconds, so the checks are either sampled
 outputs it computes one by one or properties that hold at any size:
@@ -32,7 +38,8 @@ from second_order_post_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-WL = "llama3_70b_down_8192x28672"
+WORKLOADS = ["llama3_70b_down_8192x28672", "llama2_7b_attn_4096",
+             "llama2_7b_mlp_up_11008x4096", "llama2_7b_mlp_down_4096x11008"]
 
 
 def _rows_matvec(M, v, col_scale=None, row_scale=None, chunk=2048):
@@ -50,11 +57,12 @@ def _rows_matvec(M, v, col_scale=None, row_scale=None, chunk=2048):
     return out
 
 
-@pytest.fixture(scope="module")
-def run(cuda_device):
+@pytest.fixture(scope="module", params=WORKLOADS)
+def run(cuda_device, request):
     from second_order_post_b200 import kronq as K
     from second_order_post_b200.engine import SublayerEngine
-    wl = synth.WORKLOADS[WL]
+    torch.cuda.empty_cache()
+    wl = synth.WORKLOADS[request.param]
     data = synth.make_workload(wl, device="cuda")
     W, X, G = data["W"], data["X"], data["G"]
     eng = SublayerEngine(wl.d_out, wl.d_in, bits=wl.bits, group=wl.group,
