@@ -217,6 +217,77 @@ def workload_config(wl, args):
             "parallelism": f"{args.gpus} independent sublayers, one per GPU"}
 
 
+# ---------------------------------------------------------------- model stack
+def run_stack(args, spec):
+    """One step = the whole stack: every covariance and score, the bit
+    allocation, every sublayer quantized at its width. Inputs are generated
+    per layer on the device (outside the timed spans); the device time is the
+    sum of CUDA-event spans around the library calls."""
+    import torch
+
+    from second_order_post_b200 import kronq as K
+    from second_order_post_b200 import synth
+    from second_order_post_b200.stack import StackEngine, device_ms, stack_flops
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("the stack workload runs on one GPU")
+    torch.cuda.set_device(0)
+    se = StackEngine(spec)
+    for _ in range(args.warmup):
+        se.run()
+    torch.cuda.synchronize()
+    se.check_info()
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(0).uuid)
+    cov_spans, q_spans, totals = [], [], []
+    l0 = K.kronq_kernel_launches()
+    with ClockSampler(uuid) as clk:
+        for _ in range(args.steps):
+            c, q = [], []
+            for layer in range(spec.layers):
+                se.score_layer(layer, timer=c)
+            bits = se.allocate()
+            S = len(se.HG[0])
+            for layer in range(spec.layers):
+                for si in range(S):
+                    se.quantize_sublayer(layer, si, bits[layer * S + si], timer=q)
+            torch.cuda.synchronize()
+            cov_spans.append(device_ms(c))
+            q_spans.append(device_ms(q))
+            totals.append(cov_spans[-1] + q_spans[-1])
+    launches = (K.kronq_kernel_launches() - l0) // args.steps
+    se.check_info()
+    ms = statistics.mean(totals)
+    flops = stack_flops(spec)
+    n = spec.n
+    cov_flops = spec.layers * (sum(n * d * (d + 1) for _, d in synth.STACK_X_GROUPS) +
+                               sum(n * do * (do + 1) for _, do, _, _ in synth.STACK_SUBLAYERS))
+    peaks, peak_src = load_peaks()
+    cov_ms = statistics.mean(cov_spans)
+    achieved = cov_flops / (cov_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    hist = [bits.count(b) for b in (2, 3, 4)]
+    line = {
+        "metric": METRIC, "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16+f32", "data": "synthetic",
+        "config": {"workload": spec.name, "layers": spec.layers,
+                   "sublayers": spec.layers * len(synth.STACK_SUBLAYERS),
+                   "tokens_per_sublayer": n, "budget_bits": spec.budget,
+                   "bits_histogram_2_3_4": hist,
+                   "l2": "inputs larger than L2", "parallelism": "1 GPU"},
+        "roofline": {"kernel": "cov_bf16 (all covariances of the stack)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 sustained"},
+        "cpu_baseline": None, "e2e": None, "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "steps_ms": {"covariances_and_scores": cov_ms,
+                     "biip_chol_obs_all_sublayers": statistics.mean(q_spans)},
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- our engine
 def main():
     ap = argparse.ArgumentParser()
@@ -231,6 +302,13 @@ def main():
     args = ap.parse_args()
 
     from second_order_post_b200 import synth
+    if args.workload in synth.STACKS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the oracle arm is timed on the single-sublayer workloads"}))
+            return
+        run_stack(args, synth.STACKS[args.workload])
+        return
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)

@@ -1106,6 +1106,136 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
   }
 }
 
+// ------------------------------------------------------------- large Q_m
+// For 32 < m (the 172 of 11008 = 64 * 172) the Q_m mix is a small GEMM per
+// group, Y = Q X, and runs as one: Qᵀ stays in shared memory for the life of
+// a persistent CTA (one per SM) and each thread accumulates a 4 x 4 tile of
+// outputs, two 16-byte shared loads per 16 FMA.
+constexpr int QB_THREADS = 256;
+constexpr int QB_CW = 64;                 // columns per work item (column side)
+constexpr int QB_SMEM_FLOATS = 227 * 1024 / 4;
+
+__device__ void load_qt(float *Qt, const float *Q, int m, int mp) {
+  for (int e = threadIdx.x; e < mp * mp; e += QB_THREADS) {
+    const int k = e / mp, b = e % mp;
+    Qt[e] = (k < m && b < m) ? Q[b * m + k] : 0.f;
+  }
+}
+
+// Column side: each group of m consecutive rows of M (R x C, in place) is
+// replaced by Q_m times it; work items are (group, 64-column tile).
+__global__ void __launch_bounds__(QB_THREADS, 1)
+    qmix_rows_kernel(float *M, int64_t ld, int64_t C, int m, int64_t groups,
+                     const float *Q) {
+  extern __shared__ float4 qb_sm4[];
+  const int mp = (m + 3) & ~3, nb4 = mp / 4;
+  float *Qt = reinterpret_cast<float *>(qb_sm4);
+  float4 *Qt4 = qb_sm4;
+  float4 *X4 = qb_sm4 + mp * nb4;           // [mp][QB_CW / 4]
+  constexpr int NC4 = QB_CW / 4;
+  load_qt(Qt, Q, m, mp);
+  const int64_t ctiles = (C + QB_CW - 1) / QB_CW;
+  const int64_t items = groups * ctiles;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int64_t a = item / ctiles, c0 = (item % ctiles) * QB_CW;
+    float *base = M + a * m * ld;
+    __syncthreads();
+    for (int e4 = threadIdx.x; e4 < mp * NC4; e4 += QB_THREADS) {
+      const int k = e4 / NC4, c4 = e4 % NC4;
+      const int64_t col = c0 + 4 * c4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k < m && col < C) v = *reinterpret_cast<const float4 *>(base + k * ld + col);
+      X4[e4] = v;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < nb4 * NC4; t += QB_THREADS) {
+      const int b4 = t / NC4, c4 = t % NC4;
+      float4 acc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < m; ++k) {
+        const float4 q = Qt4[k * nb4 + b4], x = X4[k * NC4 + c4];
+        const float qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i].x = fmaf(qq[i], x.x, acc[i].x);
+          acc[i].y = fmaf(qq[i], x.y, acc[i].y);
+          acc[i].z = fmaf(qq[i], x.z, acc[i].z);
+          acc[i].w = fmaf(qq[i], x.w, acc[i].w);
+        }
+      }
+      const int64_t col = c0 + 4 * c4;
+      if (col < C) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int b = 4 * b4 + i;
+          if (b < m) *reinterpret_cast<float4 *>(base + b * ld + col) = acc[i];
+        }
+      }
+    }
+  }
+}
+
+// Row pass for 32 < m: work items are row chunks of L*m contiguous columns:
+// load with the factors, Hadamard over a in shared memory, then
+// Y[a][b] = sum_k X[a][k] Q[b][k] written straight to global memory.
+__global__ void __launch_bounds__(QB_THREADS, 1) row_big_kernel(RowP p, int64_t items) {
+  extern __shared__ float4 qb_sm4[];
+  const int m = p.m, L = p.L, mp = (m + 3) & ~3, nb4 = mp / 4;
+  const int CH = L * m;
+  float *Qt = reinterpret_cast<float *>(qb_sm4);
+  const float4 *Qt4 = qb_sm4;
+  float *X = Qt + mp * mp;
+  load_qt(Qt, p.Q, m, mp);
+  auto vb = [](int v) { return v; };
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int64_t row = item / p.chunks, c0 = (item % p.chunks) * CH;
+    const float rf = p.norm * (p.cr ? p.cr[row] : 1.f);
+    __syncthreads();
+    for (int e = threadIdx.x; e < CH; e += QB_THREADS) {
+      float v = load_in(p.in, p.in_bf16, row * p.ld_in + c0 + e) * rf;
+      if (p.cc) v *= p.cc[c0 + e];
+      X[e] = v;
+    }
+    __syncthreads();
+    fwht_rest(X, m, L, 1, m, vb);
+    float *o = p.out + row * p.ld_out + c0;
+    const int na4 = (L + 3) / 4;
+    for (int t = threadIdx.x; t < na4 * nb4; t += QB_THREADS) {
+      const int a4 = t / nb4, b4 = t % nb4;
+      float4 acc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int a0 = 4 * a4;
+      const float *x0 = X + a0 * m;
+      for (int k = 0; k < m; ++k) {
+        const float4 q = Qt4[k * nb4 + b4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float xv = a0 + i < L ? x0[i * m + k] : 0.f;
+          acc[i].x = fmaf(xv, q.x, acc[i].x);
+          acc[i].y = fmaf(xv, q.y, acc[i].y);
+          acc[i].z = fmaf(xv, q.z, acc[i].z);
+          acc[i].w = fmaf(xv, q.w, acc[i].w);
+        }
+      }
+      const int b0 = 4 * b4;
+      if (b0 < m) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (a0 + i < L) *reinterpret_cast<float4 *>(o + (a0 + i) * m + b0) = acc[i];
+      }
+    }
+  }
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
 // ------------------------------------------------------------- planning
 struct SideRot {
   int64_t d, had, m;
@@ -1167,7 +1297,15 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
   const int64_t had_c = sc.rot ? sc.had : 1, m_c = sc.rot ? sc.m : 1;
   // ---- row pass over chunks of Lc * m_c contiguous columns
   int64_t Lc = 1;
-  if (sc.rot) {
+  const int64_t mpc = (m_c + 3) / 4 * 4;
+  // large Q_m on the column side: the persistent GEMM-style row pass, whose
+  // shared memory holds Q_mᵀ next to the chunk
+  const bool big = sc.rot && m_c > 32 && m_c % 4 == 0 && ld_out % 4 == 0 &&
+                   reinterpret_cast<uintptr_t>(out) % 16 == 0 &&
+                   mpc * mpc + m_c <= QB_SMEM_FLOATS;
+  if (big) {
+    while (Lc * 2 <= had_c && mpc * mpc + Lc * 2 * m_c <= QB_SMEM_FLOATS) Lc *= 2;
+  } else if (sc.rot) {
     while (Lc * 2 <= had_c && Lc * 2 * m_c <= ROW_CHUNK_MAX) Lc *= 2;
   } else {
     // no column rotation: chunks are only a unit of work
@@ -1196,8 +1334,17 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
       p.m = static_cast<int>(chunk);
       p.Q = nullptr;
     }
-    const kronq_status fast = launch_row_tpl(st, p, R, in_bf16);
-    if (fast != KRONQ_ERR_UNSUPPORTED) {
+    if (big) {
+      const int smem = static_cast<int>((mpc * mpc + chunk) * 4);
+      KQ_TRY(smem_attr(row_big_kernel, smem));
+      const int64_t items = R * p.chunks;
+      const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(items, sm_count()));
+      row_big_kernel<<<grid, QB_THREADS, smem, st>>>(p, items);
+      KQ_CHECK_LAUNCH();
+    }
+    const kronq_status fast = big ? KRONQ_OK : launch_row_tpl(st, p, R, in_bf16);
+    if (big) {
+    } else if (fast != KRONQ_ERR_UNSUPPORTED) {
       KQ_TRY(fast);
     } else {
       row_pass_kernel<<<static_cast<unsigned>(blocks), 512, smem, st>>>(p);
@@ -1215,7 +1362,18 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
   }
   // ---- otherwise two passes: Q_m over groups of m_r consecutive rows, then
   // the Hadamard
-  if (sr.rot && m_r > 1) {
+  if (sr.rot && m_r > 32 && m_r % 4 == 0 && ld_out % 4 == 0 && C % 4 == 0 &&
+      reinterpret_cast<uintptr_t>(out) % 16 == 0 &&
+      (m_r + 3) / 4 * 4 * ((m_r + 3) / 4 * 4 + QB_CW) <= QB_SMEM_FLOATS) {
+    const int mp = static_cast<int>((m_r + 3) / 4 * 4);
+    const int smem = (mp * mp + mp * QB_CW) * 4;
+    KQ_TRY(smem_attr(qmix_rows_kernel, smem));
+    const int64_t items = had_r * ceil_div(C, QB_CW);
+    const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(items, sm_count()));
+    qmix_rows_kernel<<<grid, QB_THREADS, smem, st>>>(out, ld_out, C, static_cast<int>(m_r),
+                                                     had_r, sr.Q);
+    KQ_CHECK_LAUNCH();
+  } else if (sr.rot && m_r > 1) {
     // Q_m, then Qᵀ (m <= 32) or a [m][64] input tile (m > 32)
     const size_t smem =
         (static_cast<size_t>(m_r) * m_r + (m_r > 32 ? m_r * 64 : m_r * m_r)) * 4;

@@ -85,6 +85,14 @@ class SublayerEngine:
                           stream)
         mark("cov_g")
         K.kronq_sensitivity(self.H_X, self.H_G, self.sens, stream)
+        return self.run_from_covariances(W, stream, mark)
+
+    def run_from_covariances(self, W, stream=None, mark=None, codes=None) -> QuantResult:
+        """Steps 3-5 on covariances already in H_X and H_G: BiIP, the damped
+        inverse Cholesky factor, OBS with packing. ``codes`` may replace the
+        code buffer (a narrower width than the engine was built for)."""
+        mark = mark or (lambda name: None)
+        codes = self.codes if codes is None else codes
         K.kronq_biip(self.opts, W, self.W_rot, self.H_X, self.H_G, self.s_x,
                      self.s_g, self.ws, self.info[2:3], stream)
         mark("biip")
@@ -94,18 +102,18 @@ class SublayerEngine:
             K.kronq_chol_split(self.H_X, self.opts.damp_rel, self.ws,
                                self.info[3:4], stream)
             mark("chol")
-            K.kronq_quantize_split(self.opts, self.W_rot, self.H_X, self.codes,
+            K.kronq_quantize_split(self.opts, self.W_rot, self.H_X, codes,
                                    self.scales, self.zeros, self.ws,
                                    self.info[4:5], stream)
         else:
             K.kronq_chol_inv(self.H_X, self.opts.damp_rel, self.ws, self.info[3:4],
                              stream)
             mark("chol")
-            K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, self.codes,
+            K.kronq_quantize_sublayer(self.opts, self.W_rot, self.H_X, codes,
                                       self.scales, self.zeros, self.ws,
                                       self.info[4:5], stream)
         mark("quant")
-        return QuantResult(self.codes, self.scales, self.zeros, self.W_rot,
+        return QuantResult(codes, self.scales, self.zeros, self.W_rot,
                            self.s_x, self.s_g, self.sens)
 
     def check_info(self):

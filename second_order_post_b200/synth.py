@@ -143,3 +143,80 @@ def make_spd(d, seed=0, cond_spread=2.0, device="cpu"):
     s = log_uniform(d, -cond_spread / 2, cond_spread / 2, gen, device)
     b = b * s[:, None]
     return (b @ b.T / k).to(torch.float32)
+
+
+# ---------------------------------------------------------------- 7B stack
+# A LLaMA-2-7B-shaped stack: per layer the sublayers q, k, v, o (4096 x 4096),
+# gate, up (11008 x 4096) and down (4096 x 11008). q, k and v read the same
+# input X, and so do gate and up; o and down have their own. Every sublayer
+# has its own output gradients G. Each layer draws one scale factor
+# 10^U(-1, 1) per tensor kind (W, X, G) that multiplies all of that layer's
+# tensors of the kind; within a tensor the recipes of the single-sublayer
+# workloads apply (attention W with 4 input columns x30, the down input
+# Student-t).
+STACK_SUBLAYERS = (
+    # name, d_out, d_in, input group
+    ("q", 4096, 4096, "attn"),
+    ("k", 4096, 4096, "attn"),
+    ("v", 4096, 4096, "attn"),
+    ("o", 4096, 4096, "o"),
+    ("gate", 11008, 4096, "mlp"),
+    ("up", 11008, 4096, "mlp"),
+    ("down", 4096, 11008, "down"),
+)
+STACK_X_GROUPS = (("attn", 4096), ("o", 4096), ("mlp", 4096), ("down", 11008))
+
+
+@dataclasses.dataclass(frozen=True)
+class StackSpec:
+    name: str = "llama2_7b_stack_224"
+    layers: int = 32
+    n: int = 32768          # calibration tokens per sublayer
+    budget: float = 3.0     # average bits
+    group: int = 128
+    damp_rel: float = 0.01
+    seed: int = 0
+
+
+STACKS = {"llama2_7b_stack_224": StackSpec()}
+
+
+def stack_rotation(d):
+    """(had, m) of a stack dimension: powers of two rotate with m = 1, 11008
+    as Hadamard-64 x Q_172."""
+    return (64, 172) if d == 11008 else (d, 1)
+
+
+def stack_layer_factors(spec: StackSpec, layer: int):
+    """(f_W, f_X, f_G): the layer's scale factor per tensor kind."""
+    gen = _gen("cpu", spec.seed + 5000 + layer)
+    f = torch.pow(10.0, -1.0 + 2.0 * torch.rand(3, generator=gen, dtype=torch.float64))
+    return tuple(float(x) for x in f)
+
+
+def make_stack_x(spec: StackSpec, layer: int, gi: int, device="cpu"):
+    name, d = STACK_X_GROUPS[gi]
+    fx = stack_layer_factors(spec, layer)[1]
+    x = make_activations(spec.n, d, -1.0, 1.0, torch.float32, device,
+                         seed=spec.seed + 200000 + 100 * layer + gi,
+                         student_t=(name == "down"))
+    return (x * fx).to(torch.bfloat16)
+
+
+def make_stack_g(spec: StackSpec, layer: int, si: int, device="cpu"):
+    d_out = STACK_SUBLAYERS[si][1]
+    fg = stack_layer_factors(spec, layer)[2]
+    g = make_activations(spec.n, d_out, -4.0, 0.0, torch.float32, device,
+                         seed=spec.seed + 300000 + 100 * layer + si)
+    return (g * fg).to(torch.bfloat16)
+
+
+def make_stack_w(spec: StackSpec, layer: int, si: int, device="cpu"):
+    name, d_out, d_in, group = STACK_SUBLAYERS[si]
+    attn = group in ("attn", "o")
+    wl = Workload(f"{spec.name}.{layer}.{name}", d_out, d_in, spec.n, torch.bfloat16,
+                  2, spec.group, stack_rotation(d_in), stack_rotation(d_out),
+                  4 if attn else 0, 30.0 if attn else 1.0)
+    fw = stack_layer_factors(spec, layer)[0]
+    w = make_weight(wl, device, seed=spec.seed + 100000 + 100 * layer + si)
+    return (w.float() * fw).to(torch.bfloat16)
