@@ -103,6 +103,31 @@ def _near_tie_pairs(scores, rel):
     return int(np.sum(np.diff(s) <= rel * s[1:]))
 
 
+def _near_tied(scores, rel):
+    """Indices whose score has a distinct neighbour closer than rel."""
+    s = np.asarray(scores)
+    out = set()
+    order = np.argsort(s)
+    for a, b in zip(order[:-1], order[1:]):
+        if s[a] != s[b] and s[b] - s[a] <= rel * s[b]:
+            out.update((int(a), int(b)))
+    return out
+
+
+def _check_allocation(got, gpu_scores, exact, numel, budget, rel):
+    """The library's bits follow the rule on its own scores exactly; against
+    the rule on the exact scores they may differ only where scores lie
+    closer than the scores' error bound (both orders are then correct)."""
+    assert list(got) == list(O.allocate_bits(gpu_scores, numel, budget))
+    want = O.allocate_bits(exact, numel, budget)
+    diff = {i for i, (g, w) in enumerate(zip(got, want)) if g != w}
+    tied = _near_tied(exact, rel)
+    if diff:
+        print(f"budget {budget}: {len(diff)} sublayers differ from the exact-score "
+              f"allocation, all within near ties: {sorted(diff)}")
+    assert diff <= tied or not diff
+
+
 def test_allocation_matches_oracle_on_exact_scores(stack):
     numel = [d_out * d_in for _ in range(SPEC.layers)
              for _, d_out, d_in, _ in synth.STACK_SUBLAYERS]
@@ -114,10 +139,7 @@ def test_allocation_matches_oracle_on_exact_scores(stack):
     ties = _near_tie_pairs(exact, 4e-4)
     print(f"stack allocation: bits histogram {np.bincount(got, minlength=5)[2:].tolist()}, "
           f"score pairs within the error bound: {ties}")
-    if ties == 0:
-        assert list(got) == list(want)
-    else:   # equal totals; differences only between near-tied scores
-        assert sum(b * m for b, m in zip(got, numel)) == sum(b * m for b, m in zip(want, numel))
+    _check_allocation(got, list(stack["sens"][:, 2]), exact, numel, SPEC.budget, 4e-4)
 
 
 def test_trx_only_allocation(stack):
@@ -128,9 +150,7 @@ def test_trx_only_allocation(stack):
     numel = se.numel(SPEC)
     got = se.allocate("trx")
     exact = stack["ex_x"]
-    want = O.allocate_bits(exact, numel, SPEC.budget)
-    if _near_tie_pairs(exact, 2e-4) == 0:
-        assert list(got) == list(want)
+    _check_allocation(got, list(stack["sens"][:, 0]), exact, numel, SPEC.budget, 2e-4)
     b = np.array(got).reshape(SPEC.layers, S)
     # the tie-break: in a layer, a later one of q/k/v never gets more bits
     assert (b[:, 0] >= b[:, 1]).all() and (b[:, 1] >= b[:, 2]).all()
@@ -158,3 +178,20 @@ def test_sampled_sublayers_replay(stack):
         w2 = w[:, h:] + ((w[:, :h] - first["w_hat"]) @ r12) @ u22
         _, bad2, _ = replay_check(w2, u22, codes[:, h:], zeros[:, gh:], bits, SPEC.group)
         assert bad1 == 0 and bad2 == 0
+
+
+@pytest.mark.parametrize("budget", [2.17, 2.6, 3.4, 3.8])
+def test_allocation_at_other_budgets(stack, budget):
+    """The greedy rule (2->3 in descending score, then 3->4) gives a mixed
+    allocation below and above 3.0 (at 3.0 every sublayer fits at 3 bits):
+    the library's bits on its own scores against the oracle allocator on the
+    exact scores."""
+    from second_order_post_b200 import kronq as K
+    numel = [d_out * d_in for _ in range(SPEC.layers)
+             for _, d_out, d_in, _ in synth.STACK_SUBLAYERS]
+    exact = stack["ex_x"] * stack["ex_g"]
+    got = K.kronq_allocate_bits(list(stack["sens"][:, 2]), numel, budget)
+    used = sum(b * m for b, m in zip(got, numel))
+    assert used <= budget * sum(numel)
+    assert len(set(got)) == 2                     # a real mix of two widths
+    _check_allocation(got, list(stack["sens"][:, 2]), exact, numel, budget, 4e-4)
