@@ -36,7 +36,7 @@ __all__ = [
     "rotation_matrix", "diag_scale", "cov", "sensitivity", "biip",
     "damping", "chol_inv", "quant_params", "obs_quantize", "rtn_quantize",
     "pack_codes", "unpack_codes", "layer_loss", "cv_rows_cols",
-    "allocate_bits",
+    "allocate_bits", "dequantize", "unrotate_matvec", "dequant_matvec",
 ]
 
 _M64 = np.uint64(0xFFFFFFFFFFFFFFFF)
@@ -307,6 +307,48 @@ def unpack_codes(words: np.ndarray, bits: int, d_in: int) -> np.ndarray:
             bit = (words[:, pos // 32] >> np.uint64(pos % 32)) & np.uint64(1)
             out[:, c] |= bit.astype(np.int64) << t
     return out
+
+
+# --------------------------------------------------------------------------
+# Using the quantized sublayer: dequantize, undo the two-sided rotation
+# [aimodeling: packed low-bit weights with a fused dequant + BiIP matvec;
+# wmrh Q2: two Hadamard transforms per layer at inference]
+# --------------------------------------------------------------------------
+def dequantize(codes, scales, zeros, group: int) -> np.ndarray:
+    """The quantizer's reconstruction: w_hat[i, c] = scale[i, g]·(q[i, c] −
+    zero[i, g]) with g = c // group (codes unpacked, d_out x d_in)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    g = np.arange(codes.shape[1]) // group
+    scales = np.asarray(scales, dtype=np.float64)
+    zeros = np.asarray(zeros, dtype=np.float64)
+    return scales[:, g] * (codes - zeros[:, g])
+
+
+def unrotate_matvec(w_rot, s_x, s_g, x, seed=0, rot_in=None, rot_out=None):
+    """y = W x for the sublayer whose rotated weights are W' = U_G S_G W S_X
+    U_Xᵀ, i.e. y = S_G⁻¹ U_Gᵀ W' U_X S_X⁻¹ x, with dense rotations built
+    from the spec. x is d_in (one token) or B x d_in (one token per row)."""
+    w_rot = np.asarray(w_rot, dtype=np.float64)
+    d_out, d_in = w_rot.shape
+    rot_in = rot_in or (d_in, 1)
+    rot_out = rot_out or (d_out, 1)
+    u_x = rotation_matrix(seed, 0, *rot_in)
+    u_g = rotation_matrix(seed, 1, *rot_out)
+    xt = np.atleast_2d(np.asarray(x, dtype=np.float64)).T          # d_in x B
+    x1 = xt / np.asarray(s_x, dtype=np.float64)[:, None]
+    y = u_g.T @ (w_rot @ (u_x @ x1))
+    y = y / np.asarray(s_g, dtype=np.float64)[:, None]
+    return y.T if np.ndim(x) == 2 else y[:, 0]
+
+
+def dequant_matvec(packed, scales, zeros, bits: int, group: int, s_x, s_g, x,
+                   seed=0, rot_in=None, rot_out=None):
+    """The quantized sublayer applied to x: unpack, dequantize, undo the
+    rotation."""
+    packed = np.asarray(packed)
+    d_in = packed.shape[1] * 32 // bits
+    w_hat = dequantize(unpack_codes(packed, bits, d_in), scales, zeros, group)
+    return unrotate_matvec(w_hat, s_x, s_g, x, seed, rot_in, rot_out)
 
 
 # --------------------------------------------------------------------------

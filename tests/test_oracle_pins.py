@@ -431,3 +431,55 @@ def test_obs_two_halves_join_through_r12():
         assert np.array_equal(np.concatenate([first["codes"], second["codes"]], 1), whole["codes"])
         assert np.allclose(np.concatenate([first["w_hat"], second["w_hat"]], 1), whole["w_hat"],
                            atol=1e-12)
+
+
+# ---------------------------------------------------------------- using the quantized layer
+def test_dequantize_hand_examples():
+    for line in open(os.path.join(GOLDEN, "dequant_examples.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        bits, sz, codes, want = (part.split() for part in line.split("|"))
+        sz = [float(v) for v in sz]
+        scales = np.array([sz[0::2]])
+        zeros = np.array([sz[1::2]])
+        codes = np.array([[int(c) for c in codes]])
+        assert max(codes[0]) < 2 ** int(bits[0])
+        got = O.dequantize(codes, scales, zeros, 4)
+        assert got.tolist() == [[float(v) for v in want]]
+
+
+@pytest.mark.parametrize("rot_out,rot_in", [((8, 3), (16, 4)), ((32, 1), (64, 1))])
+def test_unrotate_matvec_inverts_biip(rot_out, rot_in):
+    """W' = U_G S_G W S_X U_Xᵀ from the oracle's BiIP, undone: the sublayer
+    applied to x from W' equals W x (orthogonality of U, exact division by
+    the scales), for one token and for a batch."""
+    d_out, d_in = rot_out[0] * rot_out[1], rot_in[0] * rot_in[1]
+    rng = np.random.default_rng(9)
+    w = rng.standard_normal((d_out, d_in))
+    wr, _, _, sx, sg = O.biip(w, _spd(d_in, 1), _spd(d_out, 2), seed=3,
+                              rot_in=rot_in, rot_out=rot_out)
+    x = rng.standard_normal((5, d_in))
+    y = O.unrotate_matvec(wr, sx, sg, x, seed=3, rot_in=rot_in, rot_out=rot_out)
+    assert np.abs(y - x @ w.T).max() < 1e-10 * np.abs(x @ w.T).max()
+    y1 = O.unrotate_matvec(wr, sx, sg, x[2], seed=3, rot_in=rot_in, rot_out=rot_out)
+    assert np.allclose(y1, y[2], rtol=0, atol=1e-12 * np.abs(y).max())
+
+
+def test_dequant_matvec_uses_the_packed_codes():
+    """Packed codes, scales and zero points from the OBS sweep reconstruct
+    the sweep's own dequantized weights before the rotation is undone."""
+    rng = np.random.default_rng(4)
+    d_out, d_in, bits, group = 12, 256, 3, 128
+    wr = rng.standard_normal((d_out, d_in)) * 0.02
+    u = O.chol_inv(_spd(d_in, 5), 0.01)
+    res = O.obs_quantize(wr, u, bits, group)
+    assert np.array_equal(O.dequantize(res["codes"], res["scales"], res["zeros"], group),
+                          res["w_hat"])
+    packed = O.pack_codes(res["codes"], bits)
+    sx, sg = rng.uniform(0.5, 2.0, d_in), rng.uniform(0.5, 2.0, d_out)
+    x = rng.standard_normal(d_in)
+    got = O.dequant_matvec(packed, res["scales"], res["zeros"], bits, group, sx, sg, x,
+                           seed=1, rot_in=(64, 4), rot_out=(4, 3))
+    want = O.unrotate_matvec(res["w_hat"], sx, sg, x, seed=1, rot_in=(64, 4),
+                             rot_out=(4, 3))
+    assert np.array_equal(got, want)
