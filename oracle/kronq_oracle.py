@@ -324,16 +324,18 @@ def dequantize(codes, scales, zeros, group: int) -> np.ndarray:
     return scales[:, g] * (codes - zeros[:, g])
 
 
-def unrotate_matvec(w_rot, s_x, s_g, x, seed=0, rot_in=None, rot_out=None):
+def unrotate_matvec(w_rot, s_x, s_g, x, seed=0, rot_in=None, rot_out=None,
+                    no_rot_in=False, no_rot_out=False):
     """y = W x for the sublayer whose rotated weights are W' = U_G S_G W S_X
     U_Xᵀ, i.e. y = S_G⁻¹ U_Gᵀ W' U_X S_X⁻¹ x, with dense rotations built
-    from the spec. x is d_in (one token) or B x d_in (one token per row)."""
+    from the spec (a side without rotation, as in biip's flags, has U = I).
+    x is d_in (one token) or B x d_in (one token per row)."""
     w_rot = np.asarray(w_rot, dtype=np.float64)
     d_out, d_in = w_rot.shape
     rot_in = rot_in or (d_in, 1)
     rot_out = rot_out or (d_out, 1)
-    u_x = rotation_matrix(seed, 0, *rot_in)
-    u_g = rotation_matrix(seed, 1, *rot_out)
+    u_x = np.eye(d_in) if no_rot_in else rotation_matrix(seed, 0, *rot_in)
+    u_g = np.eye(d_out) if no_rot_out else rotation_matrix(seed, 1, *rot_out)
     xt = np.atleast_2d(np.asarray(x, dtype=np.float64)).T          # d_in x B
     x1 = xt / np.asarray(s_x, dtype=np.float64)[:, None]
     y = u_g.T @ (w_rot @ (u_x @ x1))

@@ -463,6 +463,14 @@ def test_unrotate_matvec_inverts_biip(rot_out, rot_in):
     assert np.abs(y - x @ w.T).max() < 1e-10 * np.abs(x @ w.T).max()
     y1 = O.unrotate_matvec(wr, sx, sg, x[2], seed=3, rot_in=rot_in, rot_out=rot_out)
     assert np.allclose(y1, y[2], rtol=0, atol=1e-12 * np.abs(y).max())
+    # one-sided BiIP (the ablation flags) undone with the same flags
+    for fi, fo in ((True, False), (False, True)):
+        wr1, _, _, sx1, sg1 = O.biip(w, _spd(d_in, 1), _spd(d_out, 2), seed=3,
+                                     rot_in=rot_in, rot_out=rot_out, no_rot_in=fi,
+                                     no_rot_out=fo)
+        y2 = O.unrotate_matvec(wr1, sx1, sg1, x, seed=3, rot_in=rot_in, rot_out=rot_out,
+                               no_rot_in=fi, no_rot_out=fo)
+        assert np.abs(y2 - x @ w.T).max() < 1e-10 * np.abs(x @ w.T).max()
 
 
 def test_dequant_matvec_uses_the_packed_codes():
