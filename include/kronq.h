@@ -354,6 +354,36 @@ kronq_status kronq_quantize_split(kronq_stream_t stream, const kronq_opts *opts,
                                   uint8_t *zeros, void *ws, size_t ws_bytes,
                                   int32_t *info_dev);
 
+/*
+ * Using the quantized sublayer [aimodeling: packed low-bit weights applied
+ * through a fused dequant + BiIP matvec; wmrh Q2: the two Hadamard transforms
+ * per layer at inference]. For n_tokens activations x (rows of an
+ * n_tokens x d_in fp32 matrix) the call computes, in the original basis,
+ *     y = S_G^-1 U_G^T W_hat' U_X S_X^-1 x      (y: n_tokens x d_out fp32)
+ * with W_hat'[i][c] = scales[i][c/group] * (q[i][c] - zeros[i][c/group]) read
+ * straight from the packed codes of kronq_quantize_sublayer (never expanded in
+ * memory), and the rotations of the spec above (opts: the same bits, group,
+ * seed, rot_in, rot_out and flags as the BiIP and OBS calls that produced the
+ * codes; s_x, s_g: the scales kronq_biip returned).
+ * kronq_matvec_prepare fills a caller-owned descriptor (device, 256-byte
+ * aligned, kronq_matvec_desc_bytes bytes) with the per-side factors sign/s
+ * and the Q_m factors once; kronq_dequant_matvec then needs a workspace of
+ * kronq_matvec_workspace_bytes(d_out, d_in, n_tokens) bytes. x, y and codes
+ * 16-byte aligned; n_tokens <= 4096 (the codes are streamed once per
+ * token, the decode case is one token). info_dev: 0 (no numerical check is
+ * made).
+ */
+size_t kronq_matvec_desc_bytes(const kronq_opts *opts, int64_t d_out, int64_t d_in);
+size_t kronq_matvec_workspace_bytes(int64_t d_out, int64_t d_in, int64_t n_tokens);
+kronq_status kronq_matvec_prepare(kronq_stream_t stream, const kronq_opts *opts,
+                                  const float *s_x, const float *s_g, int64_t d_out,
+                                  int64_t d_in, void *desc, size_t desc_bytes);
+kronq_status kronq_dequant_matvec(kronq_stream_t stream, const kronq_opts *opts,
+                                  const void *desc, const uint32_t *codes,
+                                  const float *scales, const uint8_t *zeros, int64_t d_out,
+                                  int64_t d_in, const float *x, int64_t n_tokens, float *y,
+                                  void *ws, size_t ws_bytes, int32_t *info_dev);
+
 /* Workspace bytes needed by one call (opts may be NULL except for BIIP and
  * QUANT). Returns 0 for unsupported arguments. */
 size_t kronq_workspace_bytes(kronq_ws_kind which, int64_t d_out, int64_t d_in,

@@ -215,6 +215,62 @@ kronq_status kronq_layer_loss(kronq_stream_t stream, const float *W_ref,
                     ws_bytes, info_dev);
 }
 
+size_t kronq_matvec_desc_bytes(const kronq_opts *opts, int64_t d_out, int64_t d_in) {
+  if (!opts || d_out <= 0 || d_in <= 0) return 0;
+  return matvec_desc_bytes(d_out, d_in);
+}
+
+size_t kronq_matvec_workspace_bytes(int64_t d_out, int64_t d_in, int64_t n_tokens) {
+  if (d_out <= 0 || d_in <= 0 || n_tokens <= 0) return 0;
+  return matvec_ws_bytes(d_out, d_in, n_tokens);
+}
+
+namespace {
+kronq_status check_matvec_opts(const kronq_opts *opts, int64_t d_out, int64_t d_in) {
+  if (opts->bits < 2 || opts->bits > 4) return KRONQ_ERR_INVALID_ARG;
+  if (opts->group != 32 && opts->group != 64 && opts->group != 128)
+    return KRONQ_ERR_UNSUPPORTED;
+  const bool rot_x = !(opts->flags & KRONQ_FLAG_NO_ROT_IN);
+  const bool rot_g = !(opts->flags & KRONQ_FLAG_NO_ROT_OUT);
+  if (rot_x && !rot_ok(opts->rot_in, d_in)) return KRONQ_ERR_UNSUPPORTED;
+  if (rot_g && !rot_ok(opts->rot_out, d_out)) return KRONQ_ERR_UNSUPPORTED;
+  if (d_in % opts->group || d_in % 32 || d_in > 65536 || d_out > 65536)
+    return KRONQ_ERR_UNSUPPORTED;
+  return KRONQ_OK;
+}
+}  // namespace
+
+kronq_status kronq_matvec_prepare(kronq_stream_t stream, const kronq_opts *opts,
+                                  const float *s_x, const float *s_g, int64_t d_out,
+                                  int64_t d_in, void *desc, size_t desc_bytes) {
+  if (!opts || !s_x || !s_g || !desc || d_out <= 0 || d_in <= 0) return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(check_matvec_opts(opts, d_out, d_in));
+  if (!aligned(desc, 256) || desc_bytes < matvec_desc_bytes(d_out, d_in))
+    return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  return matvec_prepare(as_stream(stream), *opts, s_x, s_g, d_out, d_in, desc);
+}
+
+kronq_status kronq_dequant_matvec(kronq_stream_t stream, const kronq_opts *opts,
+                                  const void *desc, const uint32_t *codes,
+                                  const float *scales, const uint8_t *zeros, int64_t d_out,
+                                  int64_t d_in, const float *x, int64_t n_tokens, float *y,
+                                  void *ws, size_t ws_bytes, int32_t *info_dev) {
+  if (!opts || !desc || !codes || !scales || !zeros || !x || !y || !ws || !info_dev ||
+      d_out <= 0 || d_in <= 0 || n_tokens <= 0)
+    return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(check_matvec_opts(opts, d_out, d_in));
+  if (n_tokens > 4096) return KRONQ_ERR_UNSUPPORTED;
+  if (!aligned(desc, 256) || !aligned(ws, 256) || !aligned(codes, 16) || !aligned(x, 16) ||
+      !aligned(y, 16) || ws_bytes < matvec_ws_bytes(d_out, d_in, n_tokens))
+    return KRONQ_ERR_INVALID_ARG;
+  KQ_TRY(require_sm100());
+  cudaStream_t st = as_stream(stream);
+  KQ_TRY(launch_set_int(st, info_dev, 0));
+  return dequant_matvec(st, *opts, desc, codes, scales, zeros, d_out, d_in, x, n_tokens, y, ws,
+                        info_dev);
+}
+
 kronq_status kronq_selftest_timeout(kronq_stream_t stream, uint64_t limit_ns,
                                     int32_t *info_dev) {
   if (!info_dev || limit_ns == 0 || limit_ns > kSelftestMaxNs)

@@ -1444,4 +1444,55 @@ kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
   return KRONQ_OK;
 }
 
+
+// ------------------------------------------------------------- reuse by the
+// quantized-layer matvec: one side's rotation applied along rows, and the
+// factors of both sides
+namespace {
+__global__ void side_factor_kernel(const float *s, int64_t d, int rot, uint64_t key,
+                                   float *f) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < d;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float sg = (rot && (sm64(key + static_cast<uint64_t>(i)) >> 63)) ? -1.f : 1.f;
+    f[i] = sg / s[i];
+  }
+}
+__global__ void transpose_small_kernel(const float *a, float *at, int m) {
+  for (int e = threadIdx.x; e < m * m; e += blockDim.x) at[(e % m) * m + e / m] = a[e];
+}
+}  // namespace
+
+kronq_status rotate_rows(cudaStream_t st, const float *in, float *out, int64_t R,
+                         int64_t C, bool rot, int64_t had, int64_t m, const float *Q,
+                         const float *cc, int32_t *info) {
+  const SideRot none{R, 1, 1, false, nullptr};
+  const SideRot sc{C, rot ? had : C, rot ? m : 1, rot, Q};
+  return rotate(st, in, false, C, out, C, R, C, none, sc, nullptr, cc, info);
+}
+
+kronq_status rotation_factors(cudaStream_t st, const kronq_opts &o, const float *s_x,
+                              const float *s_g, int64_t d_out, int64_t d_in, float *fx,
+                              float *fg, float *Qx, float *QgT, float *Qg, double *G) {
+  const bool rot_x = !(o.flags & KRONQ_FLAG_NO_ROT_IN);
+  const bool rot_g = !(o.flags & KRONQ_FLAG_NO_ROT_OUT);
+  const uint64_t k0 = sm64(o.seed);
+  const uint64_t kx = sm64(k0 + 0), kg = sm64(k0 + 1);
+  side_factor_kernel<<<static_cast<unsigned>(kq_min<int64_t>(ceil_div(d_in, 256), 1024)), 256,
+                       0, st>>>(s_x, d_in, rot_x, kx, fx);
+  KQ_CHECK_LAUNCH();
+  side_factor_kernel<<<static_cast<unsigned>(kq_min<int64_t>(ceil_div(d_out, 256), 1024)), 256,
+                       0, st>>>(s_g, d_out, rot_g, kg, fg);
+  KQ_CHECK_LAUNCH();
+  const uint64_t qkey = 0xA5A5A5A5A5A5A5A5ull;
+  const int mx = rot_x ? static_cast<int>(o.rot_in.m) : 1;
+  const int mg = rot_g ? static_cast<int>(o.rot_out.m) : 1;
+  QDev qx{mx, kx ^ qkey, G, Qx};
+  QDev qg{mg, kg ^ qkey, G + 256 * 256, Qg};
+  qm_kernel<<<2, 256, 0, st>>>(qx, qg);
+  KQ_CHECK_LAUNCH();
+  transpose_small_kernel<<<1, 256, 0, st>>>(Qg, QgT, mg);
+  KQ_CHECK_LAUNCH();
+  return KRONQ_OK;
+}
+
 }  // namespace kronq

@@ -76,6 +76,18 @@ kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
                   float *H_X, float *H_G, float *s_x, float *s_g, void *ws,
                   size_t ws_bytes, int32_t *info);
 
+// Rows of an R x C matrix through one side's rotation:
+// out[r] = (Hhat_had ⊗ Q_m)(cc ⊙ in[r]) / sqrt(had) (a plain cc-scaled copy
+// when rot is false; cc may be null).
+kronq_status rotate_rows(cudaStream_t st, const float *in, float *out, int64_t R,
+                         int64_t C, bool rot, int64_t had, int64_t m, const float *Q,
+                         const float *cc, int32_t *info);
+// fx = sign_x / s_x, fg = sign_g / s_g, Q_m of both sides (Qg and its
+// transpose QgT); G: 2 * 256 * 256 doubles of scratch.
+kronq_status rotation_factors(cudaStream_t st, const kronq_opts &o, const float *s_x,
+                              const float *s_g, int64_t d_out, int64_t d_in, float *fx,
+                              float *fg, float *Qx, float *QgT, float *Qg, double *G);
+
 // ---------------------------------------------------------------- OBS
 size_t quant_ws_bytes(int64_t d_out, int64_t d_in, const kronq_opts &o);
 kronq_status quantize(cudaStream_t st, const kronq_opts &o, float *W,
@@ -101,6 +113,16 @@ kronq_status quantize_split(cudaStream_t st, const kronq_opts &o, float *W,
                             const float *F, int64_t d_out, int64_t d_in, int64_t h,
                             uint32_t *codes, float *scales, uint8_t *zeros,
                             void *ws, size_t ws_bytes, int32_t *info);
+
+// ---------------------------------------------------------------- matvec
+size_t matvec_desc_bytes(int64_t d_out, int64_t d_in);
+size_t matvec_ws_bytes(int64_t d_out, int64_t d_in, int64_t B);
+kronq_status matvec_prepare(cudaStream_t st, const kronq_opts &o, const float *s_x,
+                            const float *s_g, int64_t d_out, int64_t d_in, void *desc);
+kronq_status dequant_matvec(cudaStream_t st, const kronq_opts &o, const void *desc,
+                            const uint32_t *codes, const float *scales, const uint8_t *zeros,
+                            int64_t d_out, int64_t d_in, const float *x, int64_t B, float *y,
+                            void *ws, int32_t *info);
 
 // ---------------------------------------------------------------- loss
 size_t loss_ws_bytes(int64_t d_out, int64_t d_in);

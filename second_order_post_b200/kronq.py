@@ -81,6 +81,10 @@ _SIGS = {
                                 _sz, _p],
     "kronq_layer_loss": [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _sz, _p],
     "kronq_selftest_timeout": [_p, ctypes.c_uint64, _p],
+    "kronq_matvec_desc_bytes": [_OPTS, _i64, _i64],
+    "kronq_matvec_workspace_bytes": [_i64, _i64, _i64],
+    "kronq_matvec_prepare": [_p, _OPTS, _p, _p, _i64, _i64, _p, _sz],
+    "kronq_dequant_matvec": [_p, _OPTS, _p, _p, _p, _p, _i64, _i64, _p, _i64, _p, _p, _sz, _p],
     "kronq_chol_split": [_p, _p, _i64, _f, _p, _sz, _p],
     "kronq_chol_split_point": [_i64],
     "kronq_quantize_split": [_p, _OPTS, _p, _p, _i64, _i64, _p, _p, _p, _p, _sz, _p],
@@ -98,6 +102,8 @@ for _name, _args in _SIGS.items():
     _fn.argtypes = _args
     _fn.restype = ctypes.c_int
 _lib.kronq_workspace_bytes.restype = ctypes.c_size_t
+_lib.kronq_matvec_desc_bytes.restype = ctypes.c_size_t
+_lib.kronq_matvec_workspace_bytes.restype = ctypes.c_size_t
 _lib.kronq_gemm_f32_workspace_bytes.restype = ctypes.c_size_t
 _lib.kronq_chol_split_point.restype = ctypes.c_int64
 _lib.kronq_status_string.restype = ctypes.c_char_p
@@ -207,6 +213,31 @@ def kronq_layer_loss(W_ref, W_hat, H_X, H_G, loss, ws, info, stream=None):
     _check("kronq_layer_loss", _lib.kronq_layer_loss(
         _stream(stream), _ptr(W_ref), _ptr(W_hat), _ptr(H_X), _ptr(H_G), d_out,
         d_in, _ptr(loss), _ptr(ws), ws.numel() * ws.element_size(), _ptr(info)))
+
+
+def kronq_matvec_desc_bytes(opts, d_out, d_in):
+    return int(_lib.kronq_matvec_desc_bytes(ctypes.byref(opts), d_out, d_in))
+
+
+def kronq_matvec_workspace_bytes(d_out, d_in, n_tokens):
+    return int(_lib.kronq_matvec_workspace_bytes(d_out, d_in, n_tokens))
+
+
+def kronq_matvec_prepare(opts, s_x, s_g, desc, stream=None):
+    """Fills desc (a uint8 CUDA tensor) with the factors of both sides."""
+    _check("kronq_matvec_prepare", _lib.kronq_matvec_prepare(
+        _stream(stream), ctypes.byref(opts), _ptr(s_x), _ptr(s_g), s_g.numel(),
+        s_x.numel(), _ptr(desc), desc.numel()))
+
+
+def kronq_dequant_matvec(opts, desc, codes, scales, zeros, x, y, ws, info, stream=None):
+    """y (n_tokens x d_out) = the quantized sublayer applied to x (n_tokens x d_in)."""
+    n_tokens, d_in = x.shape
+    d_out = y.shape[1]
+    _check("kronq_dequant_matvec", _lib.kronq_dequant_matvec(
+        _stream(stream), ctypes.byref(opts), _ptr(desc), _ptr(codes), _ptr(scales),
+        _ptr(zeros), d_out, d_in, _ptr(x), n_tokens, _ptr(y), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(info)))
 
 
 def kronq_selftest_timeout(limit_ns, info, stream=None):
