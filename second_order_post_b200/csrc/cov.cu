@@ -22,7 +22,11 @@
 // (the measured loss is about 0.9 ulp per MMA step of 16 rows).
 //
 // fp32 path: plain FFMA tiles (used for fp32 calibration data).
+#include <cooperative_groups.h>
+
 #include "kernels.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace kronq {
 namespace {
@@ -94,10 +98,11 @@ __global__ void __launch_bounds__(CTHREADS, 1)
   CovCtl *ctl = reinterpret_cast<CovCtl *>(smem + CSTAGES * CSTAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nt = static_cast<int>((d + CT - 1) / CT);
-  int bi, bj;
-  cov_tile(blockIdx.x, nt, bi, bj);
-  const int64_t i0 = int64_t(bi) * CT, j0 = int64_t(bj) * CT;
+  const int64_t tiles = int64_t(nt) * (nt + 1) / 2;
+  const int64_t rounds = (tiles + gridDim.x - 1) / gridDim.x;
   const int nk = static_cast<int>((n + CBK - 1) / CBK);
+  const int nchunks = nk > 0 ? (nk + CHUNK_K - 1) / CHUNK_K : 0;
+  cg::grid_group grid = cg::this_grid();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < CSTAGES; ++s) {
@@ -121,114 +126,136 @@ __global__ void __launch_bounds__(CTHREADS, 1)
   const uint32_t tbase = ctl->tmem_base;
   volatile int *abort = &ctl->abort;
 
-  int issued = 0;
-  if (warp == 0 && lane == 0) {
-    for (int it = 0; it < nk; ++it) {
-      const int s = it % CSTAGES;
-      if (it >= CSTAGES &&
-          !mbar_wait(&ctl->empty[s], ((it / CSTAGES) - 1) & 1, abort))
-        break;
-      uint8_t *st = smem + s * CSTAGE_BYTES;
-      const int32_t k0 = static_cast<int32_t>(int64_t(it) * CBK);
-      mbar_expect_tx(&ctl->full[s], CSTAGE_BYTES);
-      for (int c = 0; c < 4; ++c)
-        tma_load_2d(st + c * CBOX, &tmX, &ctl->full[s],
-                    static_cast<int32_t>(i0 + 64 * c), k0);
-      for (int c = 0; c < 4; ++c)
-        tma_load_2d(st + (4 + c) * CBOX, &tmX, &ctl->full[s],
-                    static_cast<int32_t>(j0 + 64 * c), k0);
-      issued = it + 1;
-    }
-  } else if (warp == 1 && lane == 0) {
-    // bf16 operands, both MN-major, 128 x 256 per instruction
-    const uint32_t idesc = idesc_make(1, 1, 1, 128, 256);
-    for (int it = 0; it < nk; ++it) {
-      const int s = it % CSTAGES;
-      const int ci = it / CHUNK_K, first = it % CHUNK_K == 0;
-      // a new chunk overwrites the accumulator once the last one is folded
-      if (first && ci > 0 && !mbar_wait(&ctl->folded, (ci - 1) & 1, abort)) break;
-      if (!mbar_wait(&ctl->full[s], (it / CSTAGES) & 1, abort)) break;
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(smem + s * CSTAGE_BYTES);
-      const uint32_t b0 = a0 + 4 * CBOX;
+  // Pipeline positions run on across the CTA's tiles: g counts stages
+  // (ring slot g % CSTAGES, phase g / CSTAGES), cgl counts accumulator
+  // chunks (the chunk_done / folded phases).
+  int64_t g_tma = 0, g_mma = 0;
+  int64_t cgl_mma = 0, cgl_epi = 0;
+  int64_t issued = 0;
+  for (int64_t r = 0; r < rounds; ++r) {
+    const int64_t t = blockIdx.x + r * gridDim.x;
+    if (t < tiles && !*abort) {
+      int bi, bj;
+      cov_tile(t, nt, bi, bj);
+      const int64_t i0 = int64_t(bi) * CT, j0 = int64_t(bj) * CT;
+      if (warp == 0 && lane == 0) {
+        for (int it = 0; it < nk; ++it, ++g_tma) {
+          const int s = static_cast<int>(g_tma % CSTAGES);
+          if (g_tma >= CSTAGES &&
+              !mbar_wait(&ctl->empty[s], ((g_tma / CSTAGES) - 1) & 1, abort))
+            break;
+          uint8_t *st = smem + s * CSTAGE_BYTES;
+          const int32_t k0 = static_cast<int32_t>(int64_t(it) * CBK);
+          mbar_expect_tx(&ctl->full[s], CSTAGE_BYTES);
+          for (int c = 0; c < 4; ++c)
+            tma_load_2d(st + c * CBOX, &tmX, &ctl->full[s],
+                        static_cast<int32_t>(i0 + 64 * c), k0);
+          for (int c = 0; c < 4; ++c)
+            tma_load_2d(st + (4 + c) * CBOX, &tmX, &ctl->full[s],
+                        static_cast<int32_t>(j0 + 64 * c), k0);
+          issued = g_tma + 1;
+        }
+      } else if (warp == 1 && lane == 0) {
+        // bf16 operands, both MN-major, 128 x 256 per instruction
+        const uint32_t idesc = idesc_make(1, 1, 1, 128, 256);
+        for (int it = 0; it < nk; ++it, ++g_mma) {
+          const int s = static_cast<int>(g_mma % CSTAGES);
+          const int first = it % CHUNK_K == 0;
+          // a new chunk overwrites the accumulator once the last one is folded
+          if (first) {
+            if (cgl_mma > 0 && !mbar_wait(&ctl->folded, (cgl_mma - 1) & 1, abort)) break;
+            ++cgl_mma;
+          }
+          if (!mbar_wait(&ctl->full[s], (g_mma / CSTAGES) & 1, abort)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * CSTAGE_BYTES);
+          const uint32_t b0 = a0 + 4 * CBOX;
 #pragma unroll
-      for (int kk = 0; kk < CBK / 16; ++kk) {
-        const uint64_t db = sdesc_sw128(b0 + kk * 2048, CBOX, 1024);
+          for (int kk = 0; kk < CBK / 16; ++kk) {
+            const uint64_t db = sdesc_sw128(b0 + kk * 2048, CBOX, 1024);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint64_t da = sdesc_sw128(a0 + h * 2 * CBOX + kk * 2048, CBOX, 1024);
-          umma_bf16(tbase + 256 * h, da, db, idesc, (!first || kk != 0) ? 1u : 0u);
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t da = sdesc_sw128(a0 + h * 2 * CBOX + kk * 2048, CBOX, 1024);
+              umma_bf16(tbase + 256 * h, da, db, idesc, (!first || kk != 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&ctl->empty[s]);
+          if (it % CHUNK_K == CHUNK_K - 1 || it == nk - 1) umma_commit(&ctl->chunk_done);
+          // the fold of this chunk reads the running sums (rows j of the
+          // mirror block): bring them back into L2, which the streamed rows of
+          // A evicted
+          const int ci = it / CHUNK_K;
+          const bool fold_reads = ci > 0 || beta != 0.f;
+          if (fold_reads && (it % CHUNK_K == CHUNK_K - 8 || (it == nk - 8 && nk >= 8))) {
+            const int64_t cols = kq_min<int64_t>(CT, d - i0);
+            const uint32_t bytes = static_cast<uint32_t>(cols * 4) & ~15u;
+            for (int64_t j = j0; j < kq_min<int64_t>(j0 + CT, d) && bytes > 0; ++j)
+              prefetch_l2_bulk(H + j * d + i0, bytes);
+          }
+        }
+      } else if (warp >= 2) {
+        // ---- epilogue warps: warp w folds accumulator (w-2)/4, TMEM lanes
+        // 32*(w%4) .. +31 (tile rows), all 256 columns of its half
+        const int h = (warp - 2) >> 2, q = warp & 3;
+        const int64_t i = i0 + 128 * h + 32 * q + lane;
+        const bool diag = (bi == bj);
+        for (int ci = 0; ci < nchunks; ++ci, ++cgl_epi) {
+          const bool ok = mbar_wait(&ctl->chunk_done, cgl_epi & 1, abort);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          tc_fence_after();
+          const bool last = ci == nchunks - 1;
+          for (int c = 0; c < CT / 32; ++c) {
+            float v[32];
+            tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 256 * h + 32 * c, v);
+            const int64_t jc = j0 + 32 * c;
+            if (jc >= d) continue;
+            // running sum (or the old H) at the mirror: all 32 loads before
+            // any store (their addresses are d apart, which the compiler
+            // cannot separate from the stores)
+            const bool need = ci > 0 || beta != 0.f;  // uniform across the CTA
+            const float bw = ci > 0 ? 1.f : beta;
+            float prev[32];
+            if (need) {  // unconditional loads at clamped (in-bounds) addresses
+              const int64_t ic = kq_min<int64_t>(i, d - 1);
+#pragma unroll
+              for (int tt = 0; tt < 32; ++tt)
+                prev[tt] = __ldcg(H + kq_min<int64_t>(jc + tt, d - 1) * d + ic);
+            } else {
+#pragma unroll
+              for (int tt = 0; tt < 32; ++tt) prev[tt] = 0.f;
+            }
+#pragma unroll
+            for (int tt = 0; tt < 32; ++tt) {
+              const int64_t j = jc + tt;
+              if (!((i < d) && (j < d) && (!diag || j >= i))) continue;
+              const float o = fmaf(bw, prev[tt], alpha * v[tt]);
+              H[j * d + i] = o;
+              if (last && j != i) H[i * d + j] = o;
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&ctl->folded);
         }
       }
-      umma_commit(&ctl->empty[s]);
-      if (it % CHUNK_K == CHUNK_K - 1 || it == nk - 1) umma_commit(&ctl->chunk_done);
-      // the fold of this chunk reads the running sums (rows j of the mirror
-      // block): bring them back into L2, which the streamed rows of A evicted
-      const bool fold_reads = ci > 0 || beta != 0.f;
-      if (fold_reads && (it % CHUNK_K == CHUNK_K - 8 || (it == nk - 8 && nk >= 8))) {
-        const int64_t cols = kq_min<int64_t>(CT, d - i0);
-        const uint32_t bytes = static_cast<uint32_t>(cols * 4) & ~15u;
-        for (int64_t j = j0; j < kq_min<int64_t>(j0 + CT, d) && bytes > 0; ++j)
-          prefetch_l2_bulk(H + j * d + i0, bytes);
-      }
     }
-  } else if (warp >= 2) {
-    // ---- epilogue warps: warp w folds accumulator (w-2)/4, TMEM lanes
-    // 32*(w%4) .. +31 (tile rows), all 256 columns of its half
-    const int h = (warp - 2) >> 2, q = warp & 3;
-    const int64_t i = i0 + 128 * h + 32 * q + lane;
-    const bool diag = (bi == bj);
-    const int nchunks = nk > 0 ? (nk + CHUNK_K - 1) / CHUNK_K : 0;
-    for (int ci = 0; ci < nchunks; ++ci) {
-      const bool ok = mbar_wait(&ctl->chunk_done, ci & 1, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const bool last = ci == nchunks - 1;
-      for (int c = 0; c < CT / 32; ++c) {
-        float v[32];
-        tmem_ld32(tbase + (static_cast<uint32_t>(32 * q) << 16) + 256 * h + 32 * c, v);
-        const int64_t jc = j0 + 32 * c;
-        if (jc >= d) continue;
-        // running sum (or the old H) at the mirror: all 32 loads before any
-        // store (their addresses are d apart, which the compiler cannot
-        // separate from the stores)
-        const bool need = ci > 0 || beta != 0.f;  // uniform across the CTA
-        const float bw = ci > 0 ? 1.f : beta;
-        float prev[32];
-        if (need) {  // unconditional loads at clamped (in-bounds) addresses
-          const int64_t ic = kq_min<int64_t>(i, d - 1);
-#pragma unroll
-          for (int t = 0; t < 32; ++t)
-            prev[t] = __ldcg(H + kq_min<int64_t>(jc + t, d - 1) * d + ic);
-        } else {
-#pragma unroll
-          for (int t = 0; t < 32; ++t) prev[t] = 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const int64_t j = jc + t;
-          if (!((i < d) && (j < d) && (!diag || j >= i))) continue;
-          const float o = fmaf(bw, prev[t], alpha * v[t]);
-          H[j * d + i] = o;
-          if (last && j != i) H[i * d + j] = o;
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&ctl->folded);
-    }
-    if (nchunks == 0) {  // n == 0 never reaches here (host scales H instead)
-    }
+    __syncwarp();
+    // every CTA of the grid starts the next round together, so that the
+    // tiles of a round stream the same rows of A at the same time and share
+    // them through L2 (all CTAs take the same number of barriers, also after
+    // a timeout)
+    tc_fence_before();
+    grid.sync();
+    tc_fence_after();
   }
-  __syncwarp();
 
   tc_fence_before();
   __syncthreads();
-  if (ctl->abort) {
+  if (*abort) {
     if (threadIdx.x == 0) report(info, KRONQ_ERR_TIMEOUT);
     if (warp == 0 && lane == 0) {
       const uint64_t t0 = globaltimer();
       for (int s = 0; s < CSTAGES && s < issued; ++s) {
-        const int last = ((issued - 1 - s) / CSTAGES) * CSTAGES + s;
+        const int64_t last = ((issued - 1 - s) / CSTAGES) * CSTAGES + s;
         while (!mbar_try_wait(&ctl->full[s], (last / CSTAGES) & 1) &&
                globaltimer() - t0 < kWaitLimitNs) {
         }
@@ -329,9 +356,19 @@ kronq_status cov_bf16(cudaStream_t st, const __nv_bfloat16 *A, int64_t n,
   const int64_t nt = ceil_div(d, CT);
   const int64_t tiles = nt * (nt + 1) / 2;
   KQ_TRY(smem_attr(cov_bf16_kernel, CSMEM));
-  cov_bf16_kernel<<<static_cast<unsigned>(tiles), CTHREADS, CSMEM, st>>>(
-      tm, n, d, alpha, beta, H, info);
-  KQ_CHECK_LAUNCH();
+  // persistent: one CTA per SM (the 196 KB ring allows one), all resident
+  // (cooperative launch), taking the tiles in rounds
+  int dev = 0, sms = 0, per_sm = 0;
+  KQ_CUDA(cudaGetDevice(&dev));
+  KQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  KQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, cov_bf16_kernel, CTHREADS,
+                                                        CSMEM));
+  if (per_sm < 1) return KRONQ_ERR_UNSUPPORTED;
+  const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(tiles, int64_t(sms) * per_sm));
+  void *args[] = {const_cast<CUtensorMap *>(&tm), &n, &d, &alpha, &beta, &H, &info};
+  KQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(cov_bf16_kernel), grid,
+                                      CTHREADS, args, CSMEM, st));
+  count_launch();
   return KRONQ_OK;
 }
 
