@@ -5,7 +5,9 @@
 #include <atomic>
 #include <mutex>
 #include <set>
+#include <map>
 #include <tuple>
+#include <utility>
 
 #include "kernels.cuh"
 
@@ -108,27 +110,34 @@ kronq_status require_sm100() {
 }
 
 namespace {
-// Sets a function attribute once per (device, kernel, attribute, value).
-kronq_status set_func_attr_once(const void *func, cudaFuncAttribute attr, int value) {
-  int dev = -1;
-  KQ_CUDA(cudaGetDevice(&dev));
-  static std::mutex mu;
-  static std::set<std::tuple<int, const void *, int, int>> done;
-  std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(dev, func, static_cast<int>(attr), value);
-  if (done.count(key)) return KRONQ_OK;
-  KQ_CUDA(cudaFuncSetAttribute(func, attr, value));
-  done.insert(key);
-  return KRONQ_OK;
-}
+std::mutex g_attr_mu;
 }  // namespace
 
+// The dynamic shared-memory limit of a kernel only ever rises: a launch with
+// fewer bytes than the current limit needs no change, and lowering it would
+// break a later launch of the same kernel with more.
 kronq_status set_max_dyn_smem(const void *func, int bytes) {
-  return set_func_attr_once(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  int dev = -1;
+  KQ_CUDA(cudaGetDevice(&dev));
+  static std::map<std::pair<int, const void *>, int> limit;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  int &cur = limit[std::make_pair(dev, func)];
+  if (bytes <= cur) return KRONQ_OK;
+  KQ_CUDA(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  cur = bytes;
+  return KRONQ_OK;
 }
 
 kronq_status set_nonportable_cluster(const void *func) {
-  return set_func_attr_once(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  int dev = -1;
+  KQ_CUDA(cudaGetDevice(&dev));
+  static std::set<std::pair<int, const void *>> done;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  const auto key = std::make_pair(dev, func);
+  if (done.count(key)) return KRONQ_OK;
+  KQ_CUDA(cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  done.insert(key);
+  return KRONQ_OK;
 }
 
 kronq_status make_tmap_2d(CUtensorMap *map, const void *base, bool bf16,

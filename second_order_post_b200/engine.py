@@ -73,18 +73,26 @@ class SublayerEngine:
         K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, self.info[0:1], stream)
         K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, self.info[1:2], stream)
 
-    def run(self, W, X, G, stream=None, mark=None) -> QuantResult:
+    def run(self, W, X, G, stream=None, mark=None, deps=None) -> QuantResult:
         """Enqueue the whole sublayer quantization (no host synchronisation).
         ``mark(name)``, if given, is called after each step is enqueued (the
-        benchmark records a CUDA event there)."""
+        benchmark records a CUDA event there). ``deps`` may map "cov_g" and
+        "biip" to CUDA events that the stream waits for before G and W are
+        first read (inputs still arriving on another stream)."""
         mark = mark or (lambda name: None)
+        deps = deps or {}
+        st = stream or torch.cuda.current_stream()
         K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, self.info[0:1],
                           stream)
         mark("cov_x")
+        if "cov_g" in deps:
+            st.wait_event(deps["cov_g"])
         K.kronq_accum_cov(G, self.H_G, 1.0 / G.shape[0], 0.0, self.info[1:2],
                           stream)
         mark("cov_g")
         K.kronq_sensitivity(self.H_X, self.H_G, self.sens, stream)
+        if "biip" in deps:
+            st.wait_event(deps["biip"])
         return self.run_from_covariances(W, stream, mark)
 
     def run_from_covariances(self, W, stream=None, mark=None, codes=None) -> QuantResult:
