@@ -308,7 +308,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -431,24 +431,28 @@ def main():
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         side.wait_event(e0)
-        prev_done = None
+        freed = {}   # step name -> event after the step that last reads an input
         for _ in range(args.e2e_steps):
-            # G and W cross on a side stream while X lands and H_X
-            # accumulates; the stream waits for them right before their
-            # first use (the covariance of G, BiIP)
-            if prev_done is not None:
-                side.wait_event(prev_done)
+            # the inputs cross on a copy stream, X first; each copy waits only
+            # until the previous step has finished reading that buffer, so the
+            # next X lands while this sublayer's BiIP, Cholesky and OBS run
+            arrived = {}
             with torch.cuda.stream(side):
-                Gd.copy_(Gh, non_blocking=True)
-                ev_g = torch.cuda.Event()
-                ev_g.record(side)
-                Wd.copy_(Wh, non_blocking=True)
-                ev_w = torch.cuda.Event()
-                ev_w.record(side)
-            Xd.copy_(Xh, non_blocking=True)
-            eng.run(Wd, Xd, Gd, deps={"cov_g": ev_g, "biip": ev_w})
-            prev_done = torch.cuda.Event()
-            prev_done.record(stream)
+                for key, dst, src in (("cov_x", Xd, Xh), ("cov_g", Gd, Gh), ("biip", Wd, Wh)):
+                    if key in freed:
+                        side.wait_event(freed[key])
+                    dst.copy_(src, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(side)
+                    arrived[key] = ev
+
+            def mark(name):
+                if name in ("cov_x", "cov_g", "biip"):
+                    ev = torch.cuda.Event()
+                    ev.record(stream)
+                    freed[name] = ev
+
+            eng.run(Wd, Xd, Gd, mark=mark, deps=arrived)
             codes_h.copy_(eng.codes, non_blocking=True)
             scales_h.copy_(eng.scales, non_blocking=True)
             zeros_h.copy_(eng.zeros, non_blocking=True)

@@ -76,12 +76,14 @@ class SublayerEngine:
     def run(self, W, X, G, stream=None, mark=None, deps=None) -> QuantResult:
         """Enqueue the whole sublayer quantization (no host synchronisation).
         ``mark(name)``, if given, is called after each step is enqueued (the
-        benchmark records a CUDA event there). ``deps`` may map "cov_g" and
-        "biip" to CUDA events that the stream waits for before G and W are
-        first read (inputs still arriving on another stream)."""
+        benchmark records a CUDA event there). ``deps`` may map "cov_x",
+        "cov_g" and "biip" to CUDA events that the stream waits for before X,
+        G and W are first read (inputs still arriving on another stream)."""
         mark = mark or (lambda name: None)
         deps = deps or {}
         st = stream or torch.cuda.current_stream()
+        if "cov_x" in deps:
+            st.wait_event(deps["cov_x"])
         K.kronq_accum_cov(X, self.H_X, 1.0 / X.shape[0], 0.0, self.info[0:1],
                           stream)
         mark("cov_x")
