@@ -592,6 +592,97 @@ __device__ void colpass_qmix(float *X, int AL, int m, int W4, const float *Q) {
   __syncthreads();
 }
 
+// ---- Q_28 mix on the tensor cores (warp MMA m16n8k8, TF32 in three parts)
+// fp32 accuracy from TF32 MMAs: x = hi + lo with hi, lo TF32 (rounded to
+// nearest), and a*b ~ a_hi*b_hi + a_hi*b_lo + a_lo*b_hi (the dropped a_lo*b_lo
+// is below 2^-22 |a b|).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+  hi = to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+// c (16 x 8, fp32) += a (16 x 8, tf32) * b (8 x 8, tf32); per lane (group g =
+// lane / 4, t = lane % 4): a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]},
+// b = {B[t][g], B[t+4][g]}, c = {C[g][2t], C[g][2t+1], C[g+8][2t], C[g+8][2t+1]}.
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Y = Q X for every group of 28 rows of a 16-column strip in shared memory
+// (X[(g*28 + b)*16 + c]), in place: a warp takes whole groups, Q (padded to
+// 32 x 32 with zeros) sits in registers as A fragments, the group's 28 x 16
+// block supplies the B fragments (rows 28..31 read as 0).
+__device__ void colpass_qmix_mma28(float *X, int AL, const float *Q) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  constexpr int NWARP = CP_THREADS / 32;
+  uint32_t ah[2][4][4], alo[2][4][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = mt * 16 + gq + ((e & 1) ? 8 : 0);
+        const int c = ks * 8 + tq + ((e & 2) ? 4 : 0);
+        const float q = (r < 28 && c < 28) ? __ldg(Q + r * 28 + c) : 0.f;
+        split_tf32(q, ah[mt][ks][e], alo[mt][ks][e]);
+      }
+  for (int g = warp; g < AL; g += NWARP) {
+    float *xg = X + g * 28 * 16;
+    float acc[2][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const int k0 = ks * 8 + tq, k1 = k0 + 4;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int col = nt * 8 + gq;
+        const float b0 = k0 < 28 ? xg[k0 * 16 + col] : 0.f;
+        const float b1 = k1 < 28 ? xg[k1 * 16 + col] : 0.f;
+        uint32_t b0h, b0l, b1h, b1l;
+        split_tf32(b0, b0h, b0l);
+        split_tf32(b1, b1h, b1l);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          mma_tf32(acc[mt][nt], alo[mt][ks], b0h, b1h);
+          mma_tf32(acc[mt][nt], ah[mt][ks], b0l, b1l);
+          mma_tf32(acc[mt][nt], ah[mt][ks], b0h, b1h);
+        }
+      }
+    }
+    __syncwarp();  // the whole block is read before any lane writes it
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int r0 = mt * 16 + gq, n = nt * 8 + 2 * tq;
+        if (r0 < 28)
+          *reinterpret_cast<float2 *>(xg + r0 * 16 + n) =
+              make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+        if (r0 + 8 < 28)
+          *reinterpret_cast<float2 *>(xg + (r0 + 8) * 16 + n) =
+              make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+      }
+    __syncwarp();
+  }
+  __syncthreads();
+}
+
 template <int K>
 __global__ void __launch_bounds__(CP_THREADS, 2)
     colpass_kernel(const __grid_constant__ CUtensorMap tm, ColP p) {
@@ -622,7 +713,10 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
   if (!good && threadIdx.x == 0) report(p.info, KRONQ_ERR_TIMEOUT);
   if (good) {
     // 2. Q_m over each group of m consecutive rows
-    if (m > 1) colpass_qmix(reinterpret_cast<float *>(X4), AL, m, W4, p.Q);
+    if (m == 28 && W4 == 4)
+      colpass_qmix_mma28(reinterpret_cast<float *>(X4), AL, p.Q);
+    else if (m > 1)
+      colpass_qmix(reinterpret_cast<float *>(X4), AL, m, W4, p.Q);
     // 3. Hadamard over the local bits of a (rows al*m + b, stride m rows)
     if (AL > 1) {
       int h = 1;
@@ -837,16 +931,23 @@ __device__ __forceinline__ float load1(const void *base, int64_t off) {
   else return __ldcs(reinterpret_cast<const float *>(base) + off);
 }
 
-constexpr int RT_THREADS = 512;
-
 // Row pass, one CTA per row chunk of L*M contiguous columns:
 // out = norm * cr[row] * (Hhat_L ⊗ Q_M)(cc ⊙ x) (unnormalised Hadamard times
-// norm). M == 1: vector loads into shared memory, the last Hadamard round
-// fused with the store. M > 1: the first round (radix 16) fused with the
-// loads, the Q_M mix with the store (lane b holds row b of Q_M).
+// norm). M == 1 (512 threads): vector loads into shared memory, the last
+// Hadamard round fused with the store. M == 28 (256 threads): the first round
+// (radix 32) fused with the loads; the Q_28 mix on the tensor cores on the way
+// out, Y = X Q^T with the chunk as the A operand (L x 28, row-major in shared
+// memory) and Q^T in registers as B fragments, each lane storing its pairs of
+// outputs.
+template <int M>
+struct RowThreads {
+  static constexpr int N = M == 1 ? 512 : 256;
+};
+
 template <int L, int M, bool BF16>
-__global__ void __launch_bounds__(RT_THREADS, 2) row_tpl_kernel(RowP p) {
+__global__ void __launch_bounds__(RowThreads<M>::N, 2) row_tpl_kernel(RowP p) {
   extern __shared__ float X[];
+  constexpr int NT = RowThreads<M>::N;
   constexpr int CH = L * M;
   const int64_t row = blockIdx.x / p.chunks;
   const int64_t c0 = (blockIdx.x % p.chunks) * CH;
@@ -856,7 +957,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) row_tpl_kernel(RowP p) {
   float *o = p.out + row * p.ld_out + c0;
   if constexpr (M == 1) {
     float4 *X4 = reinterpret_cast<float4 *>(X);
-    for (int e4 = threadIdx.x; e4 < CH / 4; e4 += RT_THREADS) {
+    for (int e4 = threadIdx.x; e4 < CH / 4; e4 += NT) {
       float4 v = load4<BF16>(p.in, in0 + 4 * e4);
       float4 f = make_float4(rf, rf, rf, rf);
       if (cc) {
@@ -868,8 +969,8 @@ __global__ void __launch_bounds__(RT_THREADS, 2) row_tpl_kernel(RowP p) {
     __syncthreads();
     constexpr int HL = last_round_h(L);
     constexpr int RL = L / HL;
-    trounds<L, 1, 1, HL, RT_THREADS>(X);
-    for (int t = threadIdx.x; t < L / RL; t += RT_THREADS) {
+    trounds<L, 1, 1, HL, NT>(X);
+    for (int t = threadIdx.x; t < L / RL; t += NT) {
       const int a = (t / HL) * RL * HL + (t % HL);
       float r[RL];
 #pragma unroll
@@ -879,8 +980,9 @@ __global__ void __launch_bounds__(RT_THREADS, 2) row_tpl_kernel(RowP p) {
       for (int i = 0; i < RL; ++i) o[a + i * HL] = r[i];
     }
   } else {
+    static_assert(M == 28 && L % 16 == 0, "the fixed-shape row pass takes M = 28");
     constexpr int R0 = L >= 32 ? 32 : L;
-    for (int t = threadIdx.x; t < (L / R0) * M; t += RT_THREADS) {
+    for (int t = threadIdx.x; t < (L / R0) * M; t += NT) {
       const int b = t % M, g = t / M;
       const int e0 = g * R0 * M + b;
       float r[R0];
@@ -896,32 +998,53 @@ __global__ void __launch_bounds__(RT_THREADS, 2) row_tpl_kernel(RowP p) {
       for (int i = 0; i < R0; ++i) X[e0 + i * M] = r[i];
     }
     __syncthreads();
-    trounds<L, M, R0, L, RT_THREADS>(X);
-    // Q_M mix on the way out, two groups per warp iteration
-    static_assert(M % 4 == 0 && M <= 32, "Q_M mix needs M % 4 == 0, M <= 32");
+    trounds<L, M, R0, L, NT>(X);
+    // Q_28 mix: B = Q^T (k x n) padded to 32 x 32, hi and lo parts
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int NW = RT_THREADS / 32;
-    float q[M];
+    const int gq = lane >> 2, tq = lane & 3;
+    uint32_t bh[4][4][2], bl[4][4][2];
 #pragma unroll
-    for (int k = 0; k < M; ++k) q[k] = lane < M ? __ldg(p.Q + lane * M + k) : 0.f;
-    static_assert(L % 4 == 0, "four groups per warp iteration");
-    for (int a = 4 * warp; a < L; a += 4 * NW) {
-      const float4 *x0 = reinterpret_cast<const float4 *>(X + a * M);
-      float y[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int k4 = 0; k4 < M / 4; ++k4) {
+      for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float4 u = x0[g * (M / 4) + k4];
-          y[g] = fmaf(q[4 * k4], u.x, y[g]);
-          y[g] = fmaf(q[4 * k4 + 1], u.y, y[g]);
-          y[g] = fmaf(q[4 * k4 + 2], u.z, y[g]);
-          y[g] = fmaf(q[4 * k4 + 3], u.w, y[g]);
+        for (int e = 0; e < 2; ++e) {
+          const int n = nt * 8 + gq, k = ks * 8 + tq + 4 * e;
+          const float q = (n < 28 && k < 28) ? __ldg(p.Q + n * 28 + k) : 0.f;
+          split_tf32(q, bh[nt][ks][e], bl[nt][ks][e]);
+        }
+    constexpr int NW = NT / 32;
+    for (int mt = warp; mt < L / 16; mt += NW) {
+      float acc[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+      const float *xa = X + (mt * 16 + gq) * 28;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const int k0 = ks * 8 + tq, k1 = k0 + 4;
+        uint32_t ah[4], al[4];
+        split_tf32(xa[k0], ah[0], al[0]);
+        split_tf32(xa[8 * 28 + k0], ah[1], al[1]);
+        split_tf32(k1 < 28 ? xa[k1] : 0.f, ah[2], al[2]);
+        split_tf32(k1 < 28 ? xa[8 * 28 + k1] : 0.f, ah[3], al[3]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          mma_tf32(acc[nt], al, bh[nt][ks][0], bh[nt][ks][1]);
+          mma_tf32(acc[nt], ah, bl[nt][ks][0], bl[nt][ks][1]);
+          mma_tf32(acc[nt], ah, bh[nt][ks][0], bh[nt][ks][1]);
         }
       }
-      if (lane < M) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) o[(a + g) * M + lane] = y[g];
+      for (int nt = 0; nt < 4; ++nt) {
+        const int n = nt * 8 + 2 * tq;
+        if (n < 28) {
+          const int a0 = mt * 16 + gq;
+          *reinterpret_cast<float2 *>(o + a0 * 28 + n) = make_float2(acc[nt][0], acc[nt][1]);
+          *reinterpret_cast<float2 *>(o + (a0 + 8) * 28 + n) =
+              make_float2(acc[nt][2], acc[nt][3]);
+        }
       }
     }
   }
@@ -940,7 +1063,7 @@ kronq_status launch_row_tpl(cudaStream_t st, const RowP &p, int64_t rows, bool b
   const int smem = L * M * 4;
   auto go = [&](auto kern) -> kronq_status {
     KQ_TRY(smem_attr(kern, smem));
-    kern<<<static_cast<unsigned>(blocks), RT_THREADS, smem, st>>>(p);
+    kern<<<static_cast<unsigned>(blocks), M == 1 ? 512 : 256, smem, st>>>(p);
     KQ_CHECK_LAUNCH();
     return KRONQ_OK;
   };
@@ -1029,50 +1152,10 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
   const int good = __syncthreads_and(landed);
   if (!good && threadIdx.x == 0) report(p.info, KRONQ_ERR_TIMEOUT);
   if (good) {
-    if constexpr (M > 1) {
-      // Q_M over each group of M rows: one thread per (group, column pair)
-      constexpr int W2 = 2 * W4, W = 4 * W4, M4 = M / 4;
-      static_assert(M % 4 == 0, "Q_M mix needs M % 4 == 0");
-      float *X = reinterpret_cast<float *>(X4);
-      const float4 *Q4 = reinterpret_cast<const float4 *>(p.Q);
-      for (int t = threadIdx.x; t < AL * W2; t += CP_THREADS) {
-        const int al = t / W2, c2 = t % W2;
-        float2 *base = reinterpret_cast<float2 *>(X + al * M * W) + c2;
-        float2 x[M];
-#pragma unroll
-        for (int k = 0; k < M; ++k) x[k] = base[k * W2];
-        // two output rows per step: four independent FMA chains
-#pragma unroll
-        for (int b = 0; b < M; b += 2) {
-          const float4 *q0r = Q4 + b * M4, *q1r = q0r + M4;
-          float2 y0 = make_float2(0.f, 0.f), y1 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int k4 = 0; k4 < M4; ++k4) {
-            const float4 q0 = __ldg(q0r + k4), q1 = __ldg(q1r + k4);
-            const float2 u0 = x[4 * k4], u1 = x[4 * k4 + 1];
-            const float2 u2 = x[4 * k4 + 2], u3 = x[4 * k4 + 3];
-            y0.x = fmaf(q0.x, u0.x, y0.x);
-            y0.y = fmaf(q0.x, u0.y, y0.y);
-            y1.x = fmaf(q1.x, u0.x, y1.x);
-            y1.y = fmaf(q1.x, u0.y, y1.y);
-            y0.x = fmaf(q0.y, u1.x, y0.x);
-            y0.y = fmaf(q0.y, u1.y, y0.y);
-            y1.x = fmaf(q1.y, u1.x, y1.x);
-            y1.y = fmaf(q1.y, u1.y, y1.y);
-            y0.x = fmaf(q0.z, u2.x, y0.x);
-            y0.y = fmaf(q0.z, u2.y, y0.y);
-            y1.x = fmaf(q1.z, u2.x, y1.x);
-            y1.y = fmaf(q1.z, u2.y, y1.y);
-            y0.x = fmaf(q0.w, u3.x, y0.x);
-            y0.y = fmaf(q0.w, u3.y, y0.y);
-            y1.x = fmaf(q1.w, u3.x, y1.x);
-            y1.y = fmaf(q1.w, u3.y, y1.y);
-          }
-          base[b * W2] = y0;
-          base[(b + 1) * W2] = y1;
-        }
-      }
-      __syncthreads();
+    if constexpr (M == 28) {
+      colpass_qmix_mma28(reinterpret_cast<float *>(X4), AL, p.Q);
+    } else if constexpr (M > 1) {
+      colpass_qmix(reinterpret_cast<float *>(X4), AL, M, W4, p.Q);
     }
     trounds4<AL, M * W4, 1>(X4);
   }

@@ -112,6 +112,9 @@ BIIP_CASES = [
     (688, 256, (4, 172), (256, 1), 0, torch.bfloat16),
     (344, 1376, (2, 172), (8, 172), 0, torch.float32),
     (128, 4096, (128, 1), (4096, 1), 0, torch.bfloat16),
+    # the fixed-shape row pass (Hadamard-256 x Q_28) and a 4-CTA cluster
+    # column pass with the tensor-core Q_28 mix
+    (256, 7168, (256, 1), (256, 28), 0, torch.bfloat16),
     (256, 256, (256, 1), (256, 1), 1, torch.float32),
     (256, 256, (256, 1), (256, 1), 2, torch.float32),
     (256, 256, (256, 1), (256, 1), 4, torch.float32),
