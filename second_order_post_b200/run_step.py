@@ -10,6 +10,9 @@ biip    kronq_biip on the workload's W and on symmetric positive definite
         covariances of its sizes (no covariance pass first)
 matvec  kronq_matvec_prepare + kronq_dequant_matvec on random packed codes of
         the workload's shape, one token
+chol    kronq_chol_inv on a d x d symmetric positive definite matrix
+quant   kronq_chol_inv, then kronq_quantize_sublayer of a d x d weight
+        (N(0, 0.02^2)) at 2 bits
 
 Every call goes through the C ABI; the status words are checked at the end.
 """
@@ -85,15 +88,43 @@ def run_matvec(args):
     return [info.item()]
 
 
+def run_chol(args):
+    from .engine import SublayerEngine
+    eng = SublayerEngine(args.d, args.d, bits=2, split=False)
+    H0 = _spd_like(args.d, 4, "cuda")
+    for _ in range(args.reps):
+        eng.H_X.copy_(H0)
+        K.kronq_chol_inv(eng.H_X, 0.01, eng.ws, eng.info[3:4])
+    torch.cuda.synchronize()
+    return [eng.info[3].item()]
+
+
+def run_quant(args):
+    from .engine import SublayerEngine
+    eng = SublayerEngine(args.d, args.d, bits=2, split=False)
+    eng.H_X.copy_(_spd_like(args.d, 4, "cuda"))
+    K.kronq_chol_inv(eng.H_X, 0.01, eng.ws, eng.info[3:4])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    W0 = torch.randn(args.d, args.d, generator=g, device="cuda") * 0.02
+    for _ in range(args.reps):
+        eng.W_rot.copy_(W0)
+        K.kronq_quantize_sublayer(eng.opts, eng.W_rot, eng.H_X, eng.codes, eng.scales,
+                                  eng.zeros, eng.ws, eng.info[4:5])
+    torch.cuda.synchronize()
+    return [eng.info[3].item(), eng.info[4].item()]
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("step", choices=["cov", "biip", "matvec"])
+    ap.add_argument("step", choices=["cov", "biip", "matvec", "chol", "quant"])
     ap.add_argument("--d", type=int, default=28672)
     ap.add_argument("--n", type=int, default=16384)
     ap.add_argument("--workload", default="llama3_70b_down_8192x28672")
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
-    info = {"cov": run_cov, "biip": run_biip, "matvec": run_matvec}[args.step](args)
+    info = {"cov": run_cov, "biip": run_biip, "matvec": run_matvec, "chol": run_chol,
+            "quant": run_quant}[args.step](args)
     if any(info):
         raise SystemExit(f"status word(s) {info}")
     print(f"{args.step} ok")
