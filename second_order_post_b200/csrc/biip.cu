@@ -89,7 +89,9 @@ struct QDev {
   float *Q;    // out: Q[b*m + b'] (row-major)
 };
 
-__global__ void qm_kernel(QDev a, QDev b) {
+constexpr int QM_THREADS = 1024;
+
+__global__ void __launch_bounds__(QM_THREADS) qm_kernel(QDev a, QDev b) {
   const QDev &p = blockIdx.x == 0 ? a : b;
   const int m = p.m;
   if (m <= 1) {
@@ -98,10 +100,12 @@ __global__ void qm_kernel(QDev a, QDev b) {
   }
   __shared__ double v[256];
   __shared__ double coef[256];
-  __shared__ double part[32];
-  const int nw = blockDim.x / 32, w = threadIdx.x / 32, lane = threadIdx.x & 31;
+  __shared__ double part[QM_THREADS];   // [slice][row] partial sums
+  __shared__ double red[32];
+  const int nw = QM_THREADS / 32, w = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int nsl = QM_THREADS / m;       // slices of the projection sum per row
   // Box–Muller normals: G[r][c] with t = r*m + c
-  for (int t = threadIdx.x; t < m * m; t += blockDim.x) {
+  for (int t = threadIdx.x; t < m * m; t += QM_THREADS) {
     const uint64_t x1 = sm64(p.kq + 2ull * t), x2 = sm64(p.kq + 2ull * t + 1ull);
     const double u1 = (double((x1 >> 11)) + 1.0) * 0x1.0p-53;
     const double u2 = double(x2 >> 11) * 0x1.0p-53;
@@ -109,8 +113,11 @@ __global__ void qm_kernel(QDev a, QDev b) {
     p.G[c * m + r] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
   }
   __syncthreads();
+  // classical Gram–Schmidt, each projection applied twice; the projections of
+  // a column on the earlier ones run in parallel over the earlier columns
+  // (one warp each) and the update over rows x slices of the earlier columns
   for (int j = 0; j < m; ++j) {
-    for (int r = threadIdx.x; r < m; r += blockDim.x) v[r] = p.G[j * m + r];
+    for (int r = threadIdx.x; r < m; r += QM_THREADS) v[r] = p.G[j * m + r];
     __syncthreads();
     for (int pass = 0; pass < 2; ++pass) {
       for (int i = w; i < j; i += nw) {
@@ -120,29 +127,36 @@ __global__ void qm_kernel(QDev a, QDev b) {
         if (lane == 0) coef[i] = s;
       }
       __syncthreads();
-      for (int r = threadIdx.x; r < m; r += blockDim.x) {
+      if (threadIdx.x < nsl * m) {
+        const int r = threadIdx.x % m, sl = threadIdx.x / m;
+        double s = 0.0;
+        for (int i = sl; i < j; i += nsl) s += coef[i] * p.G[i * m + r];
+        part[sl * m + r] = s;
+      }
+      __syncthreads();
+      for (int r = threadIdx.x; r < m; r += QM_THREADS) {
         double s = v[r];
-        for (int i = 0; i < j; ++i) s -= coef[i] * p.G[i * m + r];
+        for (int sl = 0; sl < nsl; ++sl) s -= part[sl * m + r];
         v[r] = s;
       }
       __syncthreads();
     }
     double s = 0.0;
-    for (int r = threadIdx.x; r < m; r += blockDim.x) s += v[r] * v[r];
+    for (int r = threadIdx.x; r < m; r += QM_THREADS) s += v[r] * v[r];
     s = warp_sum_d(s);
-    if (lane == 0) part[w] = s;
+    if (lane == 0) red[w] = s;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      double t = 0.0;
-      for (int k = 0; k < nw; ++k) t += part[k];
-      part[0] = 1.0 / sqrt(t);
+    if (threadIdx.x < 32) {
+      double t = threadIdx.x < nw ? red[threadIdx.x] : 0.0;
+      t = warp_sum_d(t);
+      if (threadIdx.x == 0) red[0] = 1.0 / sqrt(t);
     }
     __syncthreads();
-    const double inv = part[0];
-    for (int r = threadIdx.x; r < m; r += blockDim.x) p.G[j * m + r] = v[r] * inv;
+    const double inv = red[0];
+    for (int r = threadIdx.x; r < m; r += QM_THREADS) p.G[j * m + r] = v[r] * inv;
     __syncthreads();
   }
-  for (int t = threadIdx.x; t < m * m; t += blockDim.x) {
+  for (int t = threadIdx.x; t < m * m; t += QM_THREADS) {
     const int bb = t / m, bp = t % m;  // Q[b][b'] = column b', row b
     p.Q[t] = static_cast<float>(p.G[bp * m + bb]);
   }
@@ -1514,7 +1528,7 @@ kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
   const uint64_t qkey = 0xA5A5A5A5A5A5A5A5ull;
   QDev qx{rot_x ? mx : 1, sx.key ^ qkey, Gx, Qx};
   QDev qg{rot_g ? mg : 1, sg.key ^ qkey, Gg, Qg};
-  qm_kernel<<<2, 256, 0, st>>>(qx, qg);
+  qm_kernel<<<2, QM_THREADS, 0, st>>>(qx, qg);
   KQ_CHECK_LAUNCH();
 
   SideRot rx{d_in, o.rot_in.had, o.rot_in.m, rot_x, Qx};
@@ -1571,7 +1585,7 @@ kronq_status rotation_factors(cudaStream_t st, const kronq_opts &o, const float 
   const int mg = rot_g ? static_cast<int>(o.rot_out.m) : 1;
   QDev qx{mx, kx ^ qkey, G, Qx};
   QDev qg{mg, kg ^ qkey, G + 256 * 256, Qg};
-  qm_kernel<<<2, 256, 0, st>>>(qx, qg);
+  qm_kernel<<<2, QM_THREADS, 0, st>>>(qx, qg);
   KQ_CHECK_LAUNCH();
   transpose_small_kernel<<<1, 256, 0, st>>>(Qg, QgT, mg);
   KQ_CHECK_LAUNCH();
