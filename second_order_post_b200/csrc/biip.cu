@@ -81,7 +81,12 @@ __global__ void side_prep_kernel(SideDev a, SideDev b, int32_t *info) {
 }
 
 // Q_m = orthogonal factor of the seeded Gaussian m x m matrix (R diag > 0),
-// by classical Gram–Schmidt applied twice per column, in fp64. One CTA per side.
+// in fp64, one CTA per side, by block classical Gram–Schmidt with
+// reorthogonalization: for each block J of QM_NB columns,
+//   V <- (I - Q_prev Q_prevᵀ)^2 G_J        (two projection passes)
+//   V <- V R^-1, VᵀV = RᵀR (Cholesky)      (twice)
+// Every R on the way is upper triangular with a positive diagonal, so the
+// columns are those of the unique QR factor.
 struct QDev {
   int m;
   uint64_t kq;
@@ -90,6 +95,10 @@ struct QDev {
 };
 
 constexpr int QM_THREADS = 1024;
+constexpr int QM_NB = 16;                 // columns per block
+constexpr int QM_LD = QM_NB + 1;          // row stride of the blocks in shared memory
+constexpr int QM_MAX = 256;
+constexpr size_t QM_SMEM = (2 * QM_MAX * QM_LD + QM_NB * QM_LD) * sizeof(double);
 
 __global__ void __launch_bounds__(QM_THREADS) qm_kernel(QDev a, QDev b) {
   const QDev &p = blockIdx.x == 0 ? a : b;
@@ -98,12 +107,12 @@ __global__ void __launch_bounds__(QM_THREADS) qm_kernel(QDev a, QDev b) {
     if (m == 1 && threadIdx.x == 0) p.Q[0] = 1.f;
     return;
   }
-  __shared__ double v[256];
-  __shared__ double coef[256];
-  __shared__ double part[QM_THREADS];   // [slice][row] partial sums
-  __shared__ double red[32];
-  const int nw = QM_THREADS / 32, w = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int nsl = QM_THREADS / m;       // slices of the projection sum per row
+  extern __shared__ double qm_sm[];
+  double *V = qm_sm;                       // [r][c], m x QM_NB
+  double *Cm = V + QM_MAX * QM_LD;         // [i][c], projection coefficients
+  double *S = Cm + QM_MAX * QM_LD;         // [a][c], Gram matrix, then R
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  constexpr int NW = QM_THREADS / 32;
   // Box–Muller normals: G[r][c] with t = r*m + c
   for (int t = threadIdx.x; t < m * m; t += QM_THREADS) {
     const uint64_t x1 = sm64(p.kq + 2ull * t), x2 = sm64(p.kq + 2ull * t + 1ull);
@@ -113,47 +122,109 @@ __global__ void __launch_bounds__(QM_THREADS) qm_kernel(QDev a, QDev b) {
     p.G[c * m + r] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
   }
   __syncthreads();
-  // classical Gram–Schmidt, each projection applied twice; the projections of
-  // a column on the earlier ones run in parallel over the earlier columns
-  // (one warp each) and the update over rows x slices of the earlier columns
-  for (int j = 0; j < m; ++j) {
-    for (int r = threadIdx.x; r < m; r += QM_THREADS) v[r] = p.G[j * m + r];
+  for (int j0 = 0; j0 < m; j0 += QM_NB) {
+    const int nb = min(QM_NB, m - j0);
+    for (int t = threadIdx.x; t < m * QM_NB; t += QM_THREADS) {
+      const int c = t / m, r = t % m;
+      V[r * QM_LD + c] = c < nb ? p.G[(j0 + c) * m + r] : 0.0;
+    }
     __syncthreads();
-    for (int pass = 0; pass < 2; ++pass) {
-      for (int i = w; i < j; i += nw) {
-        double s = 0.0;
-        for (int r = lane; r < m; r += 32) s += p.G[i * m + r] * v[r];
-        s = warp_sum_d(s);
-        if (lane == 0) coef[i] = s;
+    for (int pass = 0; pass < 2 && j0 > 0; ++pass) {
+      // Cm = Q_prevᵀ V: a warp per earlier column i, lanes over the rows;
+      // the 16 sums are then reduced across the warp by halving, after
+      // which lane l holds the sum for column (l >> 1) & 15
+      for (int i = w; i < j0; i += NW) {
+        const double *q = p.G + static_cast<int64_t>(i) * m;
+        double acc[QM_NB];
+#pragma unroll
+        for (int c = 0; c < QM_NB; ++c) acc[c] = 0.0;
+        for (int r = lane; r < m; r += 32) {
+          const double qr = q[r];
+#pragma unroll
+          for (int c = 0; c < QM_NB; ++c) acc[c] = fma(qr, V[r * QM_LD + c], acc[c]);
+        }
+#pragma unroll
+        for (int half = QM_NB / 2, bit = 16; half >= 1; half /= 2, bit /= 2) {
+          const bool up = lane & bit;
+#pragma unroll
+          for (int k2 = 0; k2 < half; ++k2) {
+            const double send = up ? acc[k2] : acc[k2 + half];
+            const double keep = up ? acc[k2 + half] : acc[k2];
+            acc[k2] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+          }
+        }
+        acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+        if ((lane & 1) == 0) Cm[i * QM_LD + ((lane >> 1) & 15)] = acc[0];
       }
       __syncthreads();
-      if (threadIdx.x < nsl * m) {
-        const int r = threadIdx.x % m, sl = threadIdx.x / m;
-        double s = 0.0;
-        for (int i = sl; i < j; i += nsl) s += coef[i] * p.G[i * m + r];
-        part[sl * m + r] = s;
+      // V -= Q_prev Cm: a thread per (row, quarter of the columns)
+      if (threadIdx.x < 4 * m) {
+        const int cq = threadIdx.x / m, r = threadIdx.x % m;
+        double s4[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+        for (int i = 0; i < j0; ++i) {
+          const double g = p.G[static_cast<int64_t>(i) * m + r];
+          const double *cmi = Cm + i * QM_LD + 4 * cq;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) s4[c] = fma(g, cmi[c], s4[c]);
+        }
+        double *vr = V + r * QM_LD + 4 * cq;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) vr[c] -= s4[c];
       }
       __syncthreads();
+    }
+    for (int rep = 0; rep < 2; ++rep) {
+      // S = VᵀV: four threads per entry, each over every fourth row
+      {
+        const int e = threadIdx.x >> 2, sl = threadIdx.x & 3;
+        const int ra = e / QM_NB, rb = e % QM_NB;
+        double s = 0.0;
+        for (int r = sl; r < m; r += 4) s = fma(V[r * QM_LD + ra], V[r * QM_LD + rb], s);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (sl == 0) S[ra * QM_LD + rb] = s;
+      }
+      __syncthreads();
+      // S = RᵀR in place (R upper, row k of R in row k of S), one warp; the
+      // padding columns (nb..) get R = I
+      if (w == 0) {
+        const int cl = lane & 15;
+        for (int k = 0; k < QM_NB; ++k) {
+          if (k >= nb) {
+            if (lane < QM_NB) S[k * QM_LD + cl] = cl == k ? 1.0 : 0.0;
+            __syncwarp();
+            continue;
+          }
+          const double d = sqrt(S[k * QM_LD + k]);
+          __syncwarp();
+          if (lane < QM_NB && cl > k && cl < nb) S[k * QM_LD + cl] /= d;
+          if (lane == 0) S[k * QM_LD + k] = d;
+          __syncwarp();
+          // trailing update of rows k+1.. (columns > row)
+          if (lane < QM_NB && cl > k && cl < nb) {
+            const double rkc = S[k * QM_LD + cl];
+            for (int a2 = k + 1; a2 <= cl; ++a2) S[a2 * QM_LD + cl] -= S[k * QM_LD + a2] * rkc;
+          }
+          __syncwarp();
+        }
+      }
+      __syncthreads();
+      // V <- V R^-1, a thread per row (forward substitution over columns)
       for (int r = threadIdx.x; r < m; r += QM_THREADS) {
-        double s = v[r];
-        for (int sl = 0; sl < nsl; ++sl) s -= part[sl * m + r];
-        v[r] = s;
+        double *x = V + r * QM_LD;   // this thread's row, solved in place
+        for (int c = 0; c < QM_NB; ++c) {
+          double v = x[c];
+          for (int k = 0; k < c; ++k) v = fma(-x[k], S[k * QM_LD + c], v);
+          x[c] = v / S[c * QM_LD + c];
+        }
       }
       __syncthreads();
     }
-    double s = 0.0;
-    for (int r = threadIdx.x; r < m; r += QM_THREADS) s += v[r] * v[r];
-    s = warp_sum_d(s);
-    if (lane == 0) red[w] = s;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      double t = threadIdx.x < nw ? red[threadIdx.x] : 0.0;
-      t = warp_sum_d(t);
-      if (threadIdx.x == 0) red[0] = 1.0 / sqrt(t);
+    for (int t = threadIdx.x; t < m * QM_NB; t += QM_THREADS) {
+      const int c = t / m, r = t % m;
+      if (c < nb) p.G[(j0 + c) * m + r] = V[r * QM_LD + c];
     }
-    __syncthreads();
-    const double inv = red[0];
-    for (int r = threadIdx.x; r < m; r += QM_THREADS) p.G[j * m + r] = v[r] * inv;
     __syncthreads();
   }
   for (int t = threadIdx.x; t < m * m; t += QM_THREADS) {
@@ -635,10 +706,11 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
 // (X[(g*28 + b)*16 + c]), in place: a warp takes whole groups, Q (padded to
 // 32 x 32 with zeros) sits in registers as A fragments, the group's 28 x 16
 // block supplies the B fragments (rows 28..31 read as 0).
+template <int NT = CP_THREADS>
 __device__ void colpass_qmix_mma28(float *X, int AL, const float *Q) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gq = lane >> 2, tq = lane & 3;
-  constexpr int NWARP = CP_THREADS / 32;
+  constexpr int NWARP = NT / 32;
   uint32_t ah[2][4][4], alo[2][4][4];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -663,21 +735,29 @@ __device__ void colpass_qmix_mma28(float *X, int AL, const float *Q) {
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       const int k0 = ks * 8 + tq, k1 = k0 + 4;
+      uint32_t b0h[2], b0l[2], b1h[2], b1l[2];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int col = nt * 8 + gq;
         const float b0 = k0 < 28 ? xg[k0 * 16 + col] : 0.f;
         const float b1 = k1 < 28 ? xg[k1 * 16 + col] : 0.f;
-        uint32_t b0h, b0l, b1h, b1l;
-        split_tf32(b0, b0h, b0l);
-        split_tf32(b1, b1h, b1l);
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          mma_tf32(acc[mt][nt], alo[mt][ks], b0h, b1h);
-          mma_tf32(acc[mt][nt], ah[mt][ks], b0l, b1l);
-          mma_tf32(acc[mt][nt], ah[mt][ks], b0h, b1h);
-        }
+        split_tf32(b0, b0h[nt], b0l[nt]);
+        split_tf32(b1, b1h[nt], b1l[nt]);
       }
+      // the three parts in turn over all four accumulators (independent
+      // MMAs back to back)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], alo[mt][ks], b0h[nt], b1h[nt]);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], ah[mt][ks], b0l[nt], b1l[nt]);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], ah[mt][ks], b0h[nt], b1h[nt]);
     }
     __syncwarp();  // the whole block is read before any lane writes it
 #pragma unroll
@@ -1044,11 +1124,11 @@ __global__ void __launch_bounds__(RowThreads<M>::N, 2) row_tpl_kernel(RowP p) {
         split_tf32(k1 < 28 ? xa[k1] : 0.f, ah[2], al[2]);
         split_tf32(k1 < 28 ? xa[8 * 28 + k1] : 0.f, ah[3], al[3]);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          mma_tf32(acc[nt], al, bh[nt][ks][0], bh[nt][ks][1]);
-          mma_tf32(acc[nt], ah, bl[nt][ks][0], bl[nt][ks][1]);
-          mma_tf32(acc[nt], ah, bh[nt][ks][0], bh[nt][ks][1]);
-        }
+        for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[nt], al, bh[nt][ks][0], bh[nt][ks][1]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[nt], ah, bl[nt][ks][0], bl[nt][ks][1]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[nt], ah, bh[nt][ks][0], bh[nt][ks][1]);
       }
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
@@ -1064,9 +1144,147 @@ __global__ void __launch_bounds__(RowThreads<M>::N, 2) row_tpl_kernel(RowP p) {
   }
 }
 
+// Row pass for fp32 rows of L x 28 with the next rows in flight: one
+// persistent CTA per SM holds two row buffers; while one row goes through
+// the factors, the Hadamard rounds and the Q_28 mix (warp MMA, stored
+// straight to global memory), the bulk copy of a later row lands in the
+// other buffer. Qᵀ sits in registers as B fragments for the life of the CTA.
+constexpr int RP_THREADS = 512;
+int sm_count();
+
+template <int L>
+__global__ void __launch_bounds__(RP_THREADS, 1)
+    row_pipe28_kernel(RowP p, int64_t items, int32_t *info) {
+  extern __shared__ __align__(128) float rp_sm[];
+  constexpr int M = 28, CH = L * M, NT = RP_THREADS, NW = NT / 32;
+  constexpr uint32_t BYTES = CH * 4;
+  uint64_t *full = reinterpret_cast<uint64_t *>(rp_sm + 2 * CH);
+  int *abort_flag = reinterpret_cast<int *>(full + 2);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  auto src = [&](int64_t item) {
+    return static_cast<const float *>(p.in) + (item / p.chunks) * p.ld_in +
+           (item % p.chunks) * CH;
+  };
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_mbar_init();
+    for (int j = 0; j < 2; ++j) {
+      const int64_t it = blockIdx.x + j * static_cast<int64_t>(gridDim.x);
+      if (it < items) {
+        mbar_expect_tx(&full[j], BYTES);
+        bulk_load(rp_sm + j * CH, src(it), BYTES, &full[j]);
+      }
+    }
+  }
+  uint32_t bh[4][4][2], bl[4][4][2];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = nt * 8 + gq, k = ks * 8 + tq + 4 * e;
+        const float q = (n < 28 && k < 28) ? __ldg(p.Q + n * 28 + k) : 0.f;
+        split_tf32(q, bh[nt][ks][e], bl[nt][ks][e]);
+      }
+  __syncthreads();
+  int k = 0;
+  bool ok = true;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x, ++k) {
+    const int j = k & 1;
+    float *X = rp_sm + j * CH;
+    const bool landed = mbar_wait(&full[j], (k >> 1) & 1, abort_flag);
+    if (!__syncthreads_and(landed)) {
+      ok = false;
+      break;
+    }
+    const int64_t row = item / p.chunks, c0 = (item % p.chunks) * CH;
+    const float rf = p.norm * (p.cr ? p.cr[row] : 1.f);
+    const float *cc = p.cc ? p.cc + c0 : nullptr;
+    // factors and the Hadamard bits 0-4 of a
+    for (int t = threadIdx.x; t < (L / 32) * M; t += NT) {
+      const int b = t % M, g = t / M;
+      const int e0 = g * 32 * M + b;
+      float r[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int e = e0 + i * M;
+        float v = X[e] * rf;
+        if (cc) v *= __ldg(cc + e);
+        r[i] = v;
+      }
+      fwht_reg<32>(r);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) X[e0 + i * M] = r[i];
+    }
+    __syncthreads();
+    trounds<L, M, 32, L, NT>(X);
+    // Q_28 mix, Y = X Qᵀ, out by warp MMA
+    float *o = p.out + row * p.ld_out + c0;
+    for (int mt = warp; mt < L / 16; mt += NW) {
+      float acc[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+      const float *xa = X + (mt * 16 + gq) * 28;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const int k0 = ks * 8 + tq, k1 = k0 + 4;
+        uint32_t ah[4], al[4];
+        split_tf32(xa[k0], ah[0], al[0]);
+        split_tf32(xa[8 * 28 + k0], ah[1], al[1]);
+        split_tf32(k1 < 28 ? xa[k1] : 0.f, ah[2], al[2]);
+        split_tf32(k1 < 28 ? xa[8 * 28 + k1] : 0.f, ah[3], al[3]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[nt], al, bh[nt][ks][0], bh[nt][ks][1]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[nt], ah, bl[nt][ks][0], bl[nt][ks][1]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[nt], ah, bh[nt][ks][0], bh[nt][ks][1]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int n = nt * 8 + 2 * tq;
+        if (n < 28) {
+          const int a0 = mt * 16 + gq;
+          __stcs(reinterpret_cast<float2 *>(o + a0 * 28 + n), make_float2(acc[nt][0], acc[nt][1]));
+          __stcs(reinterpret_cast<float2 *>(o + (a0 + 8) * 28 + n),
+                 make_float2(acc[nt][2], acc[nt][3]));
+        }
+      }
+    }
+    __syncthreads();  // every read of this buffer is done
+    if (threadIdx.x == 0) {
+      const int64_t nx = item + 2 * static_cast<int64_t>(gridDim.x);
+      if (nx < items) {
+        fence_proxy_async_smem();
+        mbar_expect_tx(&full[j], BYTES);
+        bulk_load(X, src(nx), BYTES, &full[j]);
+      }
+    }
+  }
+  if (!ok && threadIdx.x == 0) {
+    report(info, KRONQ_ERR_TIMEOUT);
+    // copies still in flight (this iteration's and the next one's) land
+    // before the shared memory is released
+    for (int d = 0; d < 2; ++d) {
+      const int kk = k + d;
+      if (blockIdx.x + kk * static_cast<int64_t>(gridDim.x) >= items) continue;
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&full[kk & 1], (kk >> 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+}
+
 // Launches the fixed-shape row pass when (L, M, dtype) is one of the
 // compiled shapes; KRONQ_ERR_UNSUPPORTED otherwise.
-kronq_status launch_row_tpl(cudaStream_t st, const RowP &p, int64_t rows, bool bf16) {
+kronq_status launch_row_tpl(cudaStream_t st, const RowP &p, int64_t rows, bool bf16,
+                            int32_t *info) {
   const int L = p.L, M = p.m;
   if (reinterpret_cast<uintptr_t>(p.out) % 16 || p.ld_out % 4 || p.ld_in % 4 ||
       reinterpret_cast<uintptr_t>(p.in) % 16 || (p.cc && reinterpret_cast<uintptr_t>(p.cc) % 16) ||
@@ -1074,6 +1292,18 @@ kronq_status launch_row_tpl(cudaStream_t st, const RowP &p, int64_t rows, bool b
     return KRONQ_ERR_UNSUPPORTED;
   const int64_t blocks = rows * p.chunks;
   if (blocks > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
+  if (!bf16 && M == 28 && (L == 1024 || L == 512)) {
+    // fp32 rows of the Q_28 shapes: the pipelined persistent form
+    const int smem = 2 * L * M * 4 + 64;
+    const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(blocks, sm_count()));
+    auto pipe = [&](auto kern) -> kronq_status {
+      KQ_TRY(smem_attr(kern, smem));
+      kern<<<grid, RP_THREADS, smem, st>>>(p, blocks, info);
+      KQ_CHECK_LAUNCH();
+      return KRONQ_OK;
+    };
+    return L == 1024 ? pipe(row_pipe28_kernel<1024>) : pipe(row_pipe28_kernel<512>);
+  }
   const int smem = L * M * 4;
   auto go = [&](auto kern) -> kronq_status {
     KQ_TRY(smem_attr(kern, smem));
@@ -1111,10 +1341,10 @@ __host__ __device__ constexpr int colpass_box(int AL, int M) {
 
 // One Hadamard round over the local a-index of a column strip held as float4
 // vectors (V = M * 4 vectors per a).
-template <int AL, int V, int R, int H>
+template <int AL, int V, int R, int H, int NT = CP_THREADS>
 __device__ __forceinline__ void tround4(float4 *X4) {
   constexpr int T = (AL / R) * V;
-  for (int t = threadIdx.x; t < T; t += CP_THREADS) {
+  for (int t = threadIdx.x; t < T; t += NT) {
     const int v = t % V, g = t / V;
     const int a = (g / H) * R * H + (g % H);
     float4 *x = X4 + a * V + v;
@@ -1128,12 +1358,12 @@ __device__ __forceinline__ void tround4(float4 *X4) {
   __syncthreads();
 }
 
-template <int AL, int V, int H>
+template <int AL, int V, int H, int NT = CP_THREADS>
 __device__ __forceinline__ void trounds4(float4 *X4) {
   if constexpr (H < AL) {
     constexpr int R = radix_for(AL / H, 16);
-    tround4<AL, V, R, H>(X4);
-    trounds4<AL, V, H * R>(X4);
+    tround4<AL, V, R, H, NT>(X4);
+    trounds4<AL, V, H * R, NT>(X4);
   }
 }
 
@@ -1326,6 +1556,232 @@ __global__ void __launch_bounds__(QB_THREADS, 1) row_big_kernel(RowP p, int64_t 
   }
 }
 
+// ---- the same two mixes on the tensor cores (warp MMA m16n8k8, TF32 in
+// three parts, as for Q_28). The unit of work is a 32 x 16 block of the
+// product (two m tiles by two n tiles); Q_m sits in shared memory in the
+// order the fragments are read, so that a lane's values are contiguous.
+constexpr int QT_THREADS = 512;
+constexpr int QT_MAX_L = 64;              // Hadamard positions per row chunk
+
+__host__ __device__ constexpr int qt_xs_row(int m) { return (m + 7) / 8 * 8 + 4; }
+__host__ __device__ constexpr int qt_xs_col(int cw) { return cw + 8; }
+
+// C (MT*16 x NT*8) = A (MT*16 x KS*8) * B (KS*8 x NT*8) over 2 x 2 tile
+// units; loadA(mt, ks, a[4]) and loadB(nt, ks, b[2]) return fragments as
+// floats (zero outside the operands), store(mt, nt, c[4]) takes the result.
+template <class LA, class LB, class ST>
+__device__ __forceinline__ void mma3_units(int MT, int NT, int KS, LA loadA, LB loadB,
+                                           ST store) {
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  const int MP = (MT + 1) / 2, NP = (NT + 1) / 2;
+  for (int u = warp; u < MP * NP; u += nwarp) {
+    const int mt0 = 2 * (u % MP), nt0 = 2 * (u / MP);
+    const bool m1 = mt0 + 1 < MT, n1 = nt0 + 1 < NT;
+    float acc[2][2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+#pragma unroll 2
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t ah[2][4], alo[2][4], bh[2][2], bl[2][2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        if (i == 0 || m1) loadA(mt0 + i, ks, a);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split_tf32(a[e], ah[i][e], alo[i][e]);
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float b[2] = {0.f, 0.f};
+        if (j == 0 || n1) loadB(nt0 + j, ks, b);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) split_tf32(b[e], bh[j][e], bl[j][e]);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma_tf32(acc[i][j], alo[i], bh[j][0], bh[j][1]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma_tf32(acc[i][j], ah[i], bl[j][0], bl[j][1]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma_tf32(acc[i][j], ah[i], bh[j][0], bh[j][1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        if ((i == 0 || m1) && (j == 0 || n1)) store(mt0 + i, nt0 + j, acc[i][j]);
+  }
+}
+
+// Row pass for 32 < m on the tensor cores: as row_big_kernel, with the chunk
+// held as X[a][k] (row stride qt_xs_row(m), columns m.. zero) and
+// Y = X Qᵀ: B[k][n] = Q[n][k], stored per (n tile, k step, lane) as 2 floats.
+__global__ void __launch_bounds__(QT_THREADS, 1) row_big_mma_kernel(RowP p, int64_t items) {
+  extern __shared__ float4 qb_sm4[];
+  const int m = p.m, L = p.L;
+  const int KS = (m + 7) / 8, NT = KS, MT = L / 16, XS = qt_xs_row(m);
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  float *Qb = reinterpret_cast<float *>(qb_sm4);
+  float *X = Qb + NT * KS * 64;
+  for (int e = threadIdx.x; e < NT * KS * 64; e += QT_THREADS) {
+    const int f = e & 1, ln = (e >> 1) & 31, blk = e >> 6;
+    const int nt = blk / KS, ks = blk % KS;
+    const int n = nt * 8 + (ln >> 2), k = ks * 8 + (ln & 3) + 4 * f;
+    Qb[e] = (n < m && k < m) ? p.Q[n * m + k] : 0.f;
+  }
+  for (int e = threadIdx.x; e < L * (XS - m); e += QT_THREADS) {
+    const int a = e / (XS - m), k = m + e % (XS - m);
+    X[a * XS + k] = 0.f;
+  }
+  const int CH = L * m;
+  auto vb = [](int v) { return v; };
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int64_t row = item / p.chunks, c0 = (item % p.chunks) * CH;
+    const float rf = p.norm * (p.cr ? p.cr[row] : 1.f);
+    __syncthreads();
+    {
+      // four float4 loads per thread in flight (m % 4 == 0: a float4 never
+      // straddles two groups)
+      const int n4 = CH / 4;
+      const int64_t in0 = row * p.ld_in + c0;
+      const float4 *cc4 = p.cc ? reinterpret_cast<const float4 *>(p.cc + c0) : nullptr;
+      for (int e4 = threadIdx.x; e4 < n4; e4 += 4 * QT_THREADS) {
+        float4 v[4], f[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = e4 + u * QT_THREADS;
+          v[u] = f[u] = make_float4(1.f, 1.f, 1.f, 1.f);
+          if (idx < n4) {
+            v[u] = p.in_bf16 ? load4<true>(p.in, in0 + 4 * idx) : load4<false>(p.in, in0 + 4 * idx);
+            if (cc4) f[u] = __ldg(cc4 + idx);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = e4 + u * QT_THREADS;
+          if (idx < n4) {
+            const int e = 4 * idx, a = e / m, b = e - a * m;
+            *reinterpret_cast<float4 *>(X + a * XS + b) =
+                make_float4(v[u].x * rf * f[u].x, v[u].y * rf * f[u].y, v[u].z * rf * f[u].z,
+                            v[u].w * rf * f[u].w);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    fwht_rest(X, m, L, 1, XS, vb);
+    float *o = p.out + row * p.ld_out + c0;
+    mma3_units(
+        MT, NT, KS,
+        [&](int mt, int ks, float (&a)[4]) {
+          const float *x = X + (mt * 16 + gq) * XS + ks * 8 + tq;
+          a[0] = x[0];
+          a[1] = x[8 * XS];
+          a[2] = x[4];
+          a[3] = x[8 * XS + 4];
+        },
+        [&](int nt, int ks, float (&b)[2]) {
+          const float2 v = reinterpret_cast<const float2 *>(Qb)[(nt * KS + ks) * 32 + lane];
+          b[0] = v.x;
+          b[1] = v.y;
+        },
+        [&](int mt, int nt, const float (&c)[4]) {
+          const int a = mt * 16 + gq, b = nt * 8 + 2 * tq;
+          if (b < m) {
+            *reinterpret_cast<float2 *>(o + a * m + b) = make_float2(c[0], c[1]);
+            *reinterpret_cast<float2 *>(o + (a + 8) * m + b) = make_float2(c[2], c[3]);
+          }
+        });
+  }
+}
+
+// Column side for 32 < m on the tensor cores: each group of m rows of a
+// strip of CW columns, Y = Q X, with X[k][c] in shared memory (row stride
+// qt_xs_col(CW), rows m.. zero) and A[b][k] = Q[b][k] stored per (m tile,
+// k step, lane) as 4 floats.
+__global__ void __launch_bounds__(QT_THREADS, 1)
+    qmix_rows_mma_kernel(float *M, int64_t ld, int64_t C, int m, int64_t groups, int CW,
+                         const float *Q) {
+  extern __shared__ float4 qb_sm4[];
+  const int KS = (m + 7) / 8, MT = (m + 15) / 16, NT = CW / 8, XS = qt_xs_col(CW);
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  float *Qa = reinterpret_cast<float *>(qb_sm4);
+  float *X = Qa + MT * KS * 128;
+  for (int e = threadIdx.x; e < MT * KS * 128; e += QT_THREADS) {
+    const int f = e & 3, ln = (e >> 2) & 31, blk = e >> 7;
+    const int mt = blk / KS, ks = blk % KS;
+    const int b = mt * 16 + (ln >> 2) + 8 * (f & 1), k = ks * 8 + (ln & 3) + 4 * (f >> 1);
+    Qa[e] = (b < m && k < m) ? Q[b * m + k] : 0.f;
+  }
+  for (int e = threadIdx.x; e < (KS * 8 - m) * XS; e += QT_THREADS) X[m * XS + e] = 0.f;
+  const int64_t ctiles = (C + CW - 1) / CW;
+  const int64_t items = groups * ctiles;
+  const int cw4 = CW / 4;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int64_t a = item / ctiles, c0 = (item % ctiles) * CW;
+    float *base = M + a * m * ld + c0;
+    __syncthreads();
+    for (int e4 = threadIdx.x; e4 < m * cw4; e4 += 4 * QT_THREADS) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = e4 + u * QT_THREADS;
+        const int k = idx / cw4, c = 4 * (idx % cw4);
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < m * cw4 && c0 + c < C) v[u] = *reinterpret_cast<const float4 *>(base + k * ld + c);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = e4 + u * QT_THREADS;
+        const int k = idx / cw4, c = 4 * (idx % cw4);
+        if (idx < m * cw4) *reinterpret_cast<float4 *>(X + k * XS + c) = v[u];
+      }
+    }
+    __syncthreads();
+    mma3_units(
+        MT, NT, KS,
+        [&](int mt, int ks, float (&av)[4]) {
+          const float4 v = reinterpret_cast<const float4 *>(Qa)[(mt * KS + ks) * 32 + lane];
+          av[0] = v.x;
+          av[1] = v.y;
+          av[2] = v.z;
+          av[3] = v.w;
+        },
+        [&](int nt, int ks, float (&b)[2]) {
+          const float *x = X + (ks * 8 + tq) * XS + nt * 8 + gq;
+          b[0] = x[0];
+          b[1] = x[4 * XS];
+        },
+        [&](int mt, int nt, const float (&c)[4]) {
+          const int b = mt * 16 + gq, c2 = nt * 8 + 2 * tq;
+          if (c0 + c2 < C) {
+            if (b < m) *reinterpret_cast<float2 *>(base + b * ld + c2) = make_float2(c[0], c[1]);
+            if (b + 8 < m)
+              *reinterpret_cast<float2 *>(base + (b + 8) * ld + c2) = make_float2(c[2], c[3]);
+          }
+        });
+  }
+}
+
+// shared memory of the two kernels above
+size_t row_big_mma_smem(int m, int L) {
+  const size_t ks = (m + 7) / 8;
+  return (ks * ks * 64 + static_cast<size_t>(L) * qt_xs_row(m)) * 4;
+}
+size_t qmix_mma_smem(int m, int cw) {
+  const size_t ks = (m + 7) / 8, mt = (m + 15) / 16;
+  return (mt * ks * 128 + ks * 8 * qt_xs_col(cw)) * 4;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -1400,8 +1856,20 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
   const bool big = sc.rot && m_c > 32 && m_c % 4 == 0 && ld_out % 4 == 0 &&
                    reinterpret_cast<uintptr_t>(out) % 16 == 0 &&
                    mpc * mpc + m_c <= QB_SMEM_FLOATS;
+  bool big_mma = false;
   if (big) {
     while (Lc * 2 <= had_c && mpc * mpc + Lc * 2 * m_c <= QB_SMEM_FLOATS) Lc *= 2;
+    // the tensor-core form: chunks of up to QT_MAX_L Hadamard positions,
+    // whole 16-row tiles
+    const int64_t Lm = kq_min<int64_t>(had_c, QT_MAX_L);
+    const bool in_vec = reinterpret_cast<uintptr_t>(in) % 16 == 0 && ld_in % 4 == 0 &&
+                        (!cc || reinterpret_cast<uintptr_t>(cc) % 16 == 0);
+    if (in_vec && Lm % 16 == 0 &&
+        row_big_mma_smem(static_cast<int>(m_c), static_cast<int>(Lm)) <=
+            static_cast<size_t>(227 * 1024)) {
+      big_mma = true;
+      Lc = Lm;
+    }
   } else if (sc.rot) {
     while (Lc * 2 <= had_c && Lc * 2 * m_c <= ROW_CHUNK_MAX) Lc *= 2;
   } else {
@@ -1431,7 +1899,14 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
       p.m = static_cast<int>(chunk);
       p.Q = nullptr;
     }
-    if (big) {
+    if (big_mma) {
+      const int smem = static_cast<int>(row_big_mma_smem(p.m, p.L));
+      KQ_TRY(smem_attr(row_big_mma_kernel, smem));
+      const int64_t items = R * p.chunks;
+      const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(items, sm_count()));
+      row_big_mma_kernel<<<grid, QT_THREADS, smem, st>>>(p, items);
+      KQ_CHECK_LAUNCH();
+    } else if (big) {
       const int smem = static_cast<int>((mpc * mpc + chunk) * 4);
       KQ_TRY(smem_attr(row_big_kernel, smem));
       const int64_t items = R * p.chunks;
@@ -1439,7 +1914,7 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
       row_big_kernel<<<grid, QB_THREADS, smem, st>>>(p, items);
       KQ_CHECK_LAUNCH();
     }
-    const kronq_status fast = big ? KRONQ_OK : launch_row_tpl(st, p, R, in_bf16);
+    const kronq_status fast = big ? KRONQ_OK : launch_row_tpl(st, p, R, in_bf16, info);
     if (big) {
     } else if (fast != KRONQ_ERR_UNSUPPORTED) {
       KQ_TRY(fast);
@@ -1459,9 +1934,19 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
   }
   // ---- otherwise two passes: Q_m over groups of m_r consecutive rows, then
   // the Hadamard
-  if (sr.rot && m_r > 32 && m_r % 4 == 0 && ld_out % 4 == 0 && C % 4 == 0 &&
-      reinterpret_cast<uintptr_t>(out) % 16 == 0 &&
-      (m_r + 3) / 4 * 4 * ((m_r + 3) / 4 * 4 + QB_CW) <= QB_SMEM_FLOATS) {
+  const bool rows_aligned = ld_out % 4 == 0 && C % 4 == 0 &&
+                            reinterpret_cast<uintptr_t>(out) % 16 == 0;
+  if (sr.rot && m_r > 32 && m_r % 4 == 0 && rows_aligned &&
+      qmix_mma_smem(static_cast<int>(m_r), QB_CW) <= static_cast<size_t>(227 * 1024)) {
+    const int smem = static_cast<int>(qmix_mma_smem(static_cast<int>(m_r), QB_CW));
+    KQ_TRY(smem_attr(qmix_rows_mma_kernel, smem));
+    const int64_t items = had_r * ceil_div(C, QB_CW);
+    const unsigned grid = static_cast<unsigned>(kq_min<int64_t>(items, sm_count()));
+    qmix_rows_mma_kernel<<<grid, QT_THREADS, smem, st>>>(out, ld_out, C, static_cast<int>(m_r),
+                                                         had_r, QB_CW, sr.Q);
+    KQ_CHECK_LAUNCH();
+  } else if (sr.rot && m_r > 32 && m_r % 4 == 0 && rows_aligned &&
+             (m_r + 3) / 4 * 4 * ((m_r + 3) / 4 * 4 + QB_CW) <= QB_SMEM_FLOATS) {
     const int mp = static_cast<int>((m_r + 3) / 4 * 4);
     const int smem = (mp * mp + mp * QB_CW) * 4;
     KQ_TRY(smem_attr(qmix_rows_kernel, smem));
@@ -1528,7 +2013,8 @@ kronq_status biip(cudaStream_t st, const kronq_opts &o, const void *W,
   const uint64_t qkey = 0xA5A5A5A5A5A5A5A5ull;
   QDev qx{rot_x ? mx : 1, sx.key ^ qkey, Gx, Qx};
   QDev qg{rot_g ? mg : 1, sg.key ^ qkey, Gg, Qg};
-  qm_kernel<<<2, QM_THREADS, 0, st>>>(qx, qg);
+  KQ_TRY(smem_attr(qm_kernel, static_cast<int>(QM_SMEM)));
+  qm_kernel<<<2, QM_THREADS, QM_SMEM, st>>>(qx, qg);
   KQ_CHECK_LAUNCH();
 
   SideRot rx{d_in, o.rot_in.had, o.rot_in.m, rot_x, Qx};
@@ -1585,7 +2071,8 @@ kronq_status rotation_factors(cudaStream_t st, const kronq_opts &o, const float 
   const int mg = rot_g ? static_cast<int>(o.rot_out.m) : 1;
   QDev qx{mx, kx ^ qkey, G, Qx};
   QDev qg{mg, kg ^ qkey, G + 256 * 256, Qg};
-  qm_kernel<<<2, QM_THREADS, 0, st>>>(qx, qg);
+  KQ_TRY(smem_attr(qm_kernel, static_cast<int>(QM_SMEM)));
+  qm_kernel<<<2, QM_THREADS, QM_SMEM, st>>>(qx, qg);
   KQ_CHECK_LAUNCH();
   transpose_small_kernel<<<1, 256, 0, st>>>(Qg, QgT, mg);
   KQ_CHECK_LAUNCH();
