@@ -640,6 +640,9 @@ struct ColP {
   int box;          // rows per TMA box (divides the rows a CTA holds)
   const float *Q;   // m x m row-major (m > 1, m % 4 == 0), else null
   int32_t *info;
+  // diagonal factors applied on the way in (x[r][c] * fr[r] * fc[c]), null
+  // for none; only the Q_28 MMA mix applies them
+  const float *fr, *fc;
 };
 
 // y = Q x for each group of m rows, one thread per (group, column pair); x is
@@ -702,15 +705,32 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Y = Q X for every group of 28 rows of a 16-column strip in shared memory
-// (X[(g*28 + b)*16 + c]), in place: a warp takes whole groups, Q (padded to
-// 32 x 32 with zeros) sits in registers as A fragments, the group's 28 x 16
-// block supplies the B fragments (rows 28..31 read as 0).
-template <int NT = CP_THREADS>
-__device__ void colpass_qmix_mma28(float *X, int AL, const float *Q) {
+// c (16 x 8) += a (16 x 4) * b (4 x 8), TF32: a = {A[g][t], A[g+8][t]},
+// b = {B[t][g]} (the k = 4 shape, for the last 4 of 28)
+__device__ __forceinline__ void mma_tf32_k4(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k4.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+      "{%4, %5}, {%6}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// Y = Q X for every group of 28 rows of a strip of W = 8*NTN columns in
+// shared memory (X[(g*28 + b)*W + c]), in place: a warp takes whole groups,
+// Q (rows padded to 32 with zeros) sits in registers as A fragments, the
+// group's 28 x W block supplies the B fragments; k runs as three steps of 8
+// and one of 4. With fr / fc (this CTA's rows / the strip's columns) the
+// block is scaled on the way in: B = fr[g*28 + k] * X * fc[c].
+template <int NT = CP_THREADS, int NTN = 2>
+__device__ void colpass_qmix_mma28(float *X, int AL, const float *Q,
+                                   const float *fr = nullptr, const float *fc = nullptr) {
+  constexpr int W = 8 * NTN;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gq = lane >> 2, tq = lane & 3;
   constexpr int NWARP = NT / 32;
+  float fcol[NTN];
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt) fcol[nt] = fc ? __ldg(fc + nt * 8 + gq) : 1.f;
   uint32_t ah[2][4][4], alo[2][4][4];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -724,52 +744,73 @@ __device__ void colpass_qmix_mma28(float *X, int AL, const float *Q) {
         split_tf32(q, ah[mt][ks][e], alo[mt][ks][e]);
       }
   for (int g = warp; g < AL; g += NWARP) {
-    float *xg = X + g * 28 * 16;
-    float acc[2][2][4];
+    float *xg = X + g * 28 * W;
+    float acc[2][NTN][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      const int k0 = ks * 8 + tq, k1 = k0 + 4;
-      uint32_t b0h[2], b0l[2], b1h[2], b1l[2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int col = nt * 8 + gq;
-        const float b0 = k0 < 28 ? xg[k0 * 16 + col] : 0.f;
-        const float b1 = k1 < 28 ? xg[k1 * 16 + col] : 0.f;
-        split_tf32(b0, b0h[nt], b0l[nt]);
-        split_tf32(b1, b1h[nt], b1l[nt]);
+      const int k0 = ks * 8 + tq, k1 = k0 + 4;   // k1 < 28 unless ks == 3
+      uint32_t b0h[NTN], b0l[NTN], b1h[NTN], b1l[NTN];
+      float r0 = 1.f, r1 = 1.f;
+      if (fr) {
+        r0 = __ldg(fr + g * 28 + k0);
+        if (ks < 3) r1 = __ldg(fr + g * 28 + k1);
       }
-      // the three parts in turn over all four accumulators (independent
-      // MMAs back to back)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NTN; ++nt) {
+        const int col = nt * 8 + gq;
+        split_tf32(xg[k0 * W + col] * r0 * fcol[nt], b0h[nt], b0l[nt]);
+        if (ks < 3) split_tf32(xg[k1 * W + col] * r1 * fcol[nt], b1h[nt], b1l[nt]);
+      }
+      // the three parts in turn over all accumulators (independent MMAs
+      // back to back)
+      if (ks < 3) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], alo[mt][ks], b0h[nt], b1h[nt]);
+        for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+          for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], alo[mt][ks], b0h[nt], b1h[nt]);
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], ah[mt][ks], b0l[nt], b1l[nt]);
+        for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+          for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], ah[mt][ks], b0l[nt], b1l[nt]);
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], ah[mt][ks], b0h[nt], b1h[nt]);
+        for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], ah[mt][ks], b0h[nt], b1h[nt]);
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            mma_tf32_k4(acc[mt][nt], alo[mt][3][0], alo[mt][3][1], b0h[nt]);
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            mma_tf32_k4(acc[mt][nt], ah[mt][3][0], ah[mt][3][1], b0l[nt]);
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            mma_tf32_k4(acc[mt][nt], ah[mt][3][0], ah[mt][3][1], b0h[nt]);
+      }
     }
     __syncwarp();  // the whole block is read before any lane writes it
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < NTN; ++nt) {
         const int r0 = mt * 16 + gq, n = nt * 8 + 2 * tq;
         if (r0 < 28)
-          *reinterpret_cast<float2 *>(xg + r0 * 16 + n) =
+          *reinterpret_cast<float2 *>(xg + r0 * W + n) =
               make_float2(acc[mt][nt][0], acc[mt][nt][1]);
         if (r0 + 8 < 28)
-          *reinterpret_cast<float2 *>(xg + (r0 + 8) * 16 + n) =
+          *reinterpret_cast<float2 *>(xg + (r0 + 8) * W + n) =
               make_float2(acc[mt][nt][2], acc[mt][nt][3]);
       }
     __syncwarp();
@@ -808,7 +849,13 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
   if (good) {
     // 2. Q_m over each group of m consecutive rows
     if (m == 28 && W4 == 4)
-      colpass_qmix_mma28(reinterpret_cast<float *>(X4), AL, p.Q);
+      colpass_qmix_mma28<CP_THREADS, 2>(reinterpret_cast<float *>(X4), AL, p.Q,
+                                        p.fr ? p.fr + row0 : nullptr,
+                                        p.fc ? p.fc + c0 : nullptr);
+    else if (m == 28 && W4 == 2)
+      colpass_qmix_mma28<CP_THREADS, 1>(reinterpret_cast<float *>(X4), AL, p.Q,
+                                        p.fr ? p.fr + row0 : nullptr,
+                                        p.fc ? p.fc + c0 : nullptr);
     else if (m > 1)
       colpass_qmix(reinterpret_cast<float *>(X4), AL, m, W4, p.Q);
     // 3. Hadamard over the local bits of a (rows al*m + b, stride m rows)
@@ -860,7 +907,7 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
   }
 }
 
-template <int K, int M, int AL>
+template <int K, int M, int AL, int W4 = 4>
 __global__ void __launch_bounds__(CP_THREADS, 2)
     colpass_tpl_kernel(const __grid_constant__ CUtensorMap tm, ColP p);
 
@@ -868,7 +915,8 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
 // shape does not fit it (the caller then takes the two-pass route).
 kronq_status launch_colpass(cudaStream_t st, float *M, int64_t ld, int64_t R,
                             int64_t C, int64_t had, int64_t m, const float *Q,
-                            int32_t *info) {
+                            int32_t *info, const float *fr = nullptr,
+                            const float *fc = nullptr) {
   if (m > 32 || (m > 1 && (m % 4 != 0 || Q == nullptr)) || had < 1 || had * m != R)
     return KRONQ_ERR_UNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(M) % 16 || ld % 4 || C % 4)
@@ -884,6 +932,16 @@ kronq_status launch_colpass(cudaStream_t st, float *M, int64_t ld, int64_t R,
     }
   }
   if (K == 0) return KRONQ_ERR_UNSUPPORTED;
+  // Q_28 with 16-CTA clusters: 8-CTA clusters of 8-column strips fit more
+  // clusters at once (33 against 14 at 28672 rows; 5 % faster there)
+  if (m == 28 && K == 16 && W4 == 4 && R * 2 * 16 <= 8 * static_cast<int64_t>(CP_BUDGET) &&
+      C % 8 == 0) {
+    K = 8;
+    W4 = 2;
+  }
+  // factors ride on the Q_28 MMA mix of whole 16-column strips only
+  if ((fr || fc) && !(m == 28 && (W4 == 4 || W4 == 2) && C % (4 * W4) == 0))
+    return KRONQ_ERR_UNSUPPORTED;
   const int64_t strips = ceil_div(C, 4 * W4);
   if (strips * K > 0x7fffffff) return KRONQ_ERR_UNSUPPORTED;
   const int64_t AL = had / K, RK = AL * m;
@@ -903,7 +961,7 @@ kronq_status launch_colpass(cudaStream_t st, float *M, int64_t ld, int64_t R,
                       static_cast<uint32_t>(box), TMAP_NONE));
   const int smem = static_cast<int>(RK * W4 * 16 + 64);
   ColP p{M, ld, C, static_cast<int>(had), static_cast<int>(m), W4, static_cast<int>(box), Q,
-         info};
+         info, fr, fc};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(strips * K));
   cfg.blockDim = dim3(CP_THREADS);
@@ -923,6 +981,7 @@ kronq_status launch_colpass(cudaStream_t st, float *M, int64_t ld, int64_t R,
     count_launch();
     return KRONQ_OK;
   };
+  if (W4 == 2 && K == 8 && m == 28 && AL == 128) return go(colpass_tpl_kernel<8, 28, 128, 2>);
   if (W4 == 4) {  // the compiled fixed shapes
 #define KQ_COL_SHAPE(KK, MM, AA)                                              \
   if (K == KK && m == MM && AL == AA) return go(colpass_tpl_kernel<KK, MM, AA>);
@@ -1367,13 +1426,13 @@ __device__ __forceinline__ void trounds4(float4 *X4) {
   }
 }
 
-// Column pass (see colpass_kernel) with K, M and the local Hadamard length AL
-// fixed at compile time and strips of 16 columns.
-template <int K, int M, int AL>
+// Column pass (see colpass_kernel) with K, M, the local Hadamard length AL
+// and the strip width (4*W4 columns) fixed at compile time.
+template <int K, int M, int AL, int W4>
 __global__ void __launch_bounds__(CP_THREADS, 2)
     colpass_tpl_kernel(const __grid_constant__ CUtensorMap tm, ColP p) {
   extern __shared__ __align__(128) float4 X4[];
-  constexpr int W4 = 4, RK = AL * M, NV = RK * W4, BOX = colpass_box(AL, M);
+  constexpr int RK = AL * M, NV = RK * W4, BOX = colpass_box(AL, M);
   const int rank = K > 1 ? static_cast<int>(cluster_ctarank()) : 0;
   const int64_t strip = blockIdx.x / K;
   uint64_t *bar = reinterpret_cast<uint64_t *>(X4 + NV);
@@ -1397,7 +1456,10 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
   if (!good && threadIdx.x == 0) report(p.info, KRONQ_ERR_TIMEOUT);
   if (good) {
     if constexpr (M == 28) {
-      colpass_qmix_mma28(reinterpret_cast<float *>(X4), AL, p.Q);
+      static_assert(W4 == 2 || W4 == 4, "the Q_28 mix takes strips of 8 or 16 columns");
+      colpass_qmix_mma28<CP_THREADS, W4 / 2>(reinterpret_cast<float *>(X4), AL, p.Q,
+                                             p.fr ? p.fr + row0 : nullptr,
+                                             p.fc ? p.fc + c0 : nullptr);
     } else if constexpr (M > 1) {
       colpass_qmix(reinterpret_cast<float *>(X4), AL, M, W4, p.Q);
     }
@@ -1848,6 +1910,22 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
                     const float *cc, int32_t *info) {
   const int64_t had_r = sr.rot ? sr.had : 1, m_r = sr.rot ? sr.m : 1;
   const int64_t had_c = sc.rot ? sc.had : 1, m_c = sc.rot ? sc.m : 1;
+  // In place on fp32 with Q_28 on the row side, the row side goes first and
+  // takes both diagonal factors (a load per row and per column of its strip);
+  // the row pass then runs without factors (the per-element column factor
+  // would otherwise be an L2 read per element of every row).
+  bool row_side_done = false;
+  if (in == out && !in_bf16 && ld_in == ld_out && sr.rot && m_r == 28 && (cr || cc)) {
+    const kronq_status s0 =
+        launch_colpass(st, out, ld_out, R, C, had_r, m_r, sr.Q, info, cr, cc);
+    if (s0 == KRONQ_OK) {
+      row_side_done = true;
+      cr = nullptr;
+      cc = nullptr;
+    } else if (s0 != KRONQ_ERR_UNSUPPORTED) {
+      return s0;
+    }
+  }
   // ---- row pass over chunks of Lc * m_c contiguous columns
   int64_t Lc = 1;
   const int64_t mpc = (m_c + 3) / 4 * 4;
@@ -1926,6 +2004,7 @@ kronq_status rotate(cudaStream_t st, const void *in, bool in_bf16, int64_t ld_in
   // ---- column-side Hadamard bits beyond the chunk
   if (sc.rot && had_c / Lc > 1)
     KQ_TRY(launch_strided(st, out, R, ld_out, had_c / Lc, chunk, chunk));
+  if (row_side_done) return KRONQ_OK;
   // ---- row side in one pass (cluster column pass) where the shape allows
   if (sr.rot && (had_r > 1 || m_r > 1)) {
     const kronq_status s = launch_colpass(st, out, ld_out, R, C, had_r, m_r,
@@ -2045,9 +2124,108 @@ __global__ void transpose_small_kernel(const float *a, float *at, int m) {
 }
 }  // namespace
 
+// ---- a few whole rows (the tokens of a matvec): out = norm (Hhat ⊗ Q_m)
+// (cc ⊙ x) per row, each row spread over a cluster of K CTAs. CTA k holds
+// the Hadamard positions a in [k*AL, (k+1)*AL) (elements a*m + b), mixes each
+// group with Q_m, runs the Hadamard over its local a, and the top log2(K)
+// bits are one K-point Hadamard across the cluster (distributed shared
+// memory), written straight out.
+constexpr int VR_THREADS = 256;
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+template <int K>
+__global__ void __launch_bounds__(VR_THREADS)
+    vec_rot_kernel(const float *in, float *out, int64_t C, int had, int m, const float *Q,
+                   const float *cc, float norm) {
+  extern __shared__ __align__(16) float vr_sm[];
+  const int rank = K > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int64_t row = blockIdx.x / K;
+  const int AL = had / K, n = AL * m;
+  float *X = vr_sm, *Y = vr_sm + n;
+  const int64_t e0 = static_cast<int64_t>(rank) * n;
+  const float *x = in + row * C + e0;
+  for (int e = threadIdx.x; e < n; e += VR_THREADS)
+    X[e] = x[e] * norm * (cc ? __ldg(cc + e0 + e) : 1.f);
+  __syncthreads();
+  float *Z = X;
+  if (m > 1) {   // Y[a][b] = sum_k Q[b][k] X[a][k]
+    for (int t = threadIdx.x; t < n; t += VR_THREADS) {
+      const int a = t / m, b = t - a * m;
+      const float *xa = X + a * m, *qb = Q + b * m;
+      float acc = 0.f;
+      for (int k = 0; k < m; ++k) acc = fmaf(__ldg(qb + k), xa[k], acc);
+      Y[t] = acc;
+    }
+    __syncthreads();
+    Z = Y;
+  }
+  if (AL > 1) fwht_rest(Z, m, AL, 1, m, [](int v) { return v; });
+  if (K > 1) cluster_sync_all();
+  const int per = (n + K - 1) / K;
+  const uint32_t zs = smem_u32(Z);
+  for (int q = rank * per + threadIdx.x; q < min(n, (rank + 1) * per); q += VR_THREADS) {
+    float v[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+      v[j] = (K == 1 || j == rank) ? Z[q] : ld_dsmem_f32(mapa_shared(zs + 4u * q, j));
+    fwht_reg<K>(v);
+#pragma unroll
+    for (int j = 0; j < K; ++j) out[row * C + static_cast<int64_t>(j) * n + q] = v[j];
+  }
+  // no CTA leaves while another may still read its shared memory
+  if (K > 1) cluster_sync_all();
+}
+
+// Launches vec_rot_kernel when it applies (a rotation of whole rows, out not
+// aliasing in, m <= 32); KRONQ_ERR_UNSUPPORTED otherwise.
+kronq_status launch_vec_rot(cudaStream_t st, const float *in, float *out, int64_t R, int64_t C,
+                            int64_t had, int64_t m, const float *Q, const float *cc) {
+  if (R < 1 || R > 64 || in == out || m > 32 || had < 2 || had * m != C || (m > 1 && !Q))
+    return KRONQ_ERR_UNSUPPORTED;
+  const int K = static_cast<int>(kq_min<int64_t>(16, had));
+  const int64_t n = had / K * m;
+  const int smem = static_cast<int>(2 * n * 4);
+  if (smem > 48 * 1024) return KRONQ_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(R * K));
+  cfg.blockDim = dim3(VR_THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(K);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float norm = static_cast<float>(1.0 / sqrt(double(had)));
+  auto go = [&](auto kern) -> kronq_status {
+    if (K > 8) KQ_TRY(nonportable_cluster_attr(kern));
+    KQ_CUDA(cudaLaunchKernelEx(&cfg, kern, in, out, C, static_cast<int>(had), static_cast<int>(m),
+                               Q, cc, norm));
+    count_launch();
+    return KRONQ_OK;
+  };
+  switch (K) {
+    case 2: return go(vec_rot_kernel<2>);
+    case 4: return go(vec_rot_kernel<4>);
+    case 8: return go(vec_rot_kernel<8>);
+    default: return go(vec_rot_kernel<16>);
+  }
+}
+
 kronq_status rotate_rows(cudaStream_t st, const float *in, float *out, int64_t R,
                          int64_t C, bool rot, int64_t had, int64_t m, const float *Q,
                          const float *cc, int32_t *info) {
+  if (rot) {
+    const kronq_status s = launch_vec_rot(st, in, out, R, C, had, m, Q, cc);
+    if (s != KRONQ_ERR_UNSUPPORTED) return s;
+  }
   const SideRot none{R, 1, 1, false, nullptr};
   const SideRot sc{C, rot ? had : C, rot ? m : 1, rot, Q};
   return rotate(st, in, false, C, out, C, R, C, none, sc, nullptr, cc, info);

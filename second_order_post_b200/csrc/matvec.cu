@@ -122,6 +122,123 @@ __global__ void __launch_bounds__(MV_THREADS, BITS == 3 ? 1 : 2)
   }
 }
 
+// ---- 2- and 4-bit codes: two codes per packed fp32 pair instruction
+// A code q_j at bits [b*j, b*j + b) of a 16-bit half word w16 becomes a float
+// exactly as ((w16 & mask_j) | bits(2^23)) - 2^23 = q_j * 2^(b*j): no shift
+// per code. The matching x value is stored pre-scaled by 2^(-b*j) (exact), so
+// the product is q_j * x_j. Pairs of codes go through one packed subtract and
+// one packed FMA (fp32x2) into a two-lane accumulator.
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+template <int BITS>
+struct MvShapeX2 {
+  static constexpr int COLS = 32 / BITS, WORDS = 1, CHUNK = 32 * COLS;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(MV_THREADS, 2)
+    dequant_gemv_x2_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
+                           const uint8_t *__restrict__ zeros, int d_out, int d_in, int group,
+                           const float *__restrict__ x2, float *__restrict__ y1) {
+  static_assert(BITS == 2 || BITS == 4, "codes must not straddle 16-bit halves");
+  using S = MvShapeX2<BITS>;                  // one code word a lane per row
+  constexpr int PER16 = 16 / BITS;            // codes per 16-bit half word
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  constexpr uint32_t MAGIC = 0x4B000000u;     // bits of 2^23
+  __shared__ float part[MV_WARPS][MV_ROWS];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r0 = blockIdx.x * MV_ROWS;
+  const int nr = min(MV_ROWS, d_out - r0);
+  const int64_t words_row = static_cast<int64_t>(BITS) * d_in / 32;
+  const int ng = d_in / group;
+  const unsigned long long neg2 = pack2(-8388608.0f, -8388608.0f);
+  float acc[MV_ROWS];
+#pragma unroll
+  for (int k = 0; k < MV_ROWS; ++k) acc[k] = 0.f;
+  const int nchunks = (d_in + S::CHUNK - 1) / S::CHUNK;
+  for (int ch = warp; ch < nchunks; ch += MV_WARPS) {
+    const int col = ch * S::CHUNK + S::COLS * lane;
+    if (col >= d_in) continue;
+    // x pre-scaled by 2^(-BITS * position in its half word), as pairs
+    unsigned long long xp[S::COLS / 2];
+    float xsum = 0.f;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x2 + col);
+#pragma unroll
+#pragma unroll
+    for (int q = 0; q < S::COLS / 4; ++q) {
+      const float4 v = __ldg(x4 + q);
+      xsum += (v.x + v.y) + (v.z + v.w);
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j0 = 4 * q + 2 * h, j1 = j0 + 1;
+        // times 2^(-BITS * position): exact (a power of two)
+        xp[j0 / 2] = pack2(e[2 * h] * __int_as_float((127 - BITS * (j0 % PER16)) << 23),
+                           e[2 * h + 1] * __int_as_float((127 - BITS * (j1 % PER16)) << 23));
+      }
+    }
+    const int g = col / group;
+    const int64_t w0 = static_cast<int64_t>(col) * BITS / 32;
+    uint32_t w[MV_ROWS][S::WORDS];
+#pragma unroll
+    for (int k = 0; k < MV_ROWS; ++k) {
+      const int64_t row = r0 + kq_min(k, nr - 1);
+      const uint32_t *p = codes + row * words_row + w0;
+#pragma unroll
+      for (int t = 0; t < S::WORDS; ++t) w[k][t] = __ldg(p + t);
+    }
+#pragma unroll
+    for (int k = 0; k < MV_ROWS; ++k) {
+      const int64_t row = r0 + kq_min(k, nr - 1);
+      const float sc = __ldg(scales + row * ng + g);
+      const float z = static_cast<float>(__ldg(zeros + row * ng + g));
+      unsigned long long a2 = 0ull;
+#pragma unroll
+      for (int t = 0; t < S::WORDS; ++t) {
+#pragma unroll
+        for (int hw = 0; hw < 2; ++hw) {
+          const uint32_t h16 = hw ? (w[k][t] >> 16) : w[k][t];
+#pragma unroll
+          for (int i = 0; i < PER16; i += 2) {
+            const uint32_t lo = (h16 & (MASK << (BITS * i))) | MAGIC;
+            const uint32_t hi = (h16 & (MASK << (BITS * (i + 1)))) | MAGIC;
+            const int j = (t * 2 + hw) * PER16 + i;   // column within the lane's 16
+            a2 = fma2(add2(pack2(__uint_as_float(lo), __uint_as_float(hi)), neg2), xp[j / 2], a2);
+          }
+        }
+      }
+      const float dot = __uint_as_float(static_cast<uint32_t>(a2)) +
+                        __uint_as_float(static_cast<uint32_t>(a2 >> 32));
+      acc[k] = fmaf(sc, dot - z * xsum, acc[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < MV_ROWS; ++k) {
+    const float v = warp_sum(acc[k]);
+    if (lane == 0) part[warp][k] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < nr) {
+    float v = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < MV_WARPS; ++w2) v += part[w2][threadIdx.x];
+    y1[r0 + threadIdx.x] = v;
+  }
+}
+
 __global__ void scale_cols_kernel(const float *in, const float *f, float *out, int64_t B,
                                   int64_t d) {
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < B * d;
@@ -153,8 +270,13 @@ kronq_status launch_gemv(cudaStream_t st, const uint32_t *codes, const float *sc
                          const uint8_t *zeros, int64_t d_out, int64_t d_in, int group,
                          const float *x2, float *y1) {
   const int64_t grid = ceil_div(d_out, MV_ROWS);
-  dequant_gemv_kernel<BITS><<<static_cast<unsigned>(grid), MV_THREADS, 0, st>>>(
-      codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, x2, y1);
+  if constexpr (BITS == 3) {
+    dequant_gemv_kernel<BITS><<<static_cast<unsigned>(grid), MV_THREADS, 0, st>>>(
+        codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, x2, y1);
+  } else {
+    dequant_gemv_x2_kernel<BITS><<<static_cast<unsigned>(grid), MV_THREADS, 0, st>>>(
+        codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, x2, y1);
+  }
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
