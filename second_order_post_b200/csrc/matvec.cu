@@ -122,14 +122,21 @@ __global__ void __launch_bounds__(MV_THREADS, BITS == 3 ? 1 : 2)
   }
 }
 
-// ---- 2- and 4-bit codes: two codes per packed fp32 pair instruction
-// A code q_j at bits [b*j, b*j + b) of a 16-bit half word w16 becomes a float
-// exactly as ((w16 & mask_j) | bits(2^23)) - 2^23 = q_j * 2^(b*j): no shift
-// per code. The matching x value is stored pre-scaled by 2^(-b*j) (exact), so
-// the product is q_j * x_j. Pairs of codes go through one packed subtract and
-// one packed FMA (fp32x2) into a two-lane accumulator.
+// packed fp32 pairs (two lanes in one 64-bit register)
 __device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
-  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float lo_of(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float hi_of(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
 }
 __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
                                                    unsigned long long c) {
@@ -143,99 +150,125 @@ __device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigne
   return d;
 }
 
-template <int BITS>
-struct MvShapeX2 {
-  static constexpr int COLS = 32 / BITS, WORDS = 1, CHUNK = 32 * COLS;
-};
+// The streaming GEMV for 2- and 4-bit codes: every warp streams whole rows, a
+// row block of MV3_RB rows at a time, 16 bytes of code words per lane and row
+// per step (all rows' loads in flight at once); the lane's x values are read
+// once per step (L1-resident: x is the same for every row) for all the
+// block's rows.
+//   A code q at bits [b*i, b*i + b) of a 16-bit half word h becomes a float
+// exactly as ((h & mask_i) | bits(2^23)) - 2^23 = q * 2^(b*i): no shift per
+// code. x is scaled by 2^(-b*i) on the way in (exact), so the product is
+// q * x. Pairs of codes take one packed subtract and one packed FMA (fp32x2)
+// into a two-lane accumulator.
+constexpr int MV3_THREADS = 256;
+constexpr int MV3_RB = 8;                        // rows per row block of a warp
 
 template <int BITS>
-__global__ void __launch_bounds__(MV_THREADS, 2)
-    dequant_gemv_x2_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
-                           const uint8_t *__restrict__ zeros, int d_out, int d_in, int group,
-                           const float *__restrict__ x2, float *__restrict__ y1) {
-  static_assert(BITS == 2 || BITS == 4, "codes must not straddle 16-bit halves");
-  using S = MvShapeX2<BITS>;                  // one code word a lane per row
-  constexpr int PER16 = 16 / BITS;            // codes per 16-bit half word
+struct Mv3 {
+  static constexpr int WORDS = 4;                      // code words per lane and step
+  static constexpr int LCOLS = WORDS * 32 / BITS;      // columns per lane and step
+  static constexpr int TILE = 32 * LCOLS;              // columns per warp step
+};
+
+// 2^(-k) for 0 <= k <= 126, exact
+__device__ __forceinline__ float pow2_neg(int k) { return __int_as_float((127 - k) << 23); }
+
+template <int BITS>
+__global__ void __launch_bounds__(MV3_THREADS, 2)
+    dequant_gemv3_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
+                         const uint8_t *__restrict__ zeros, int d_out, int d_in, int group,
+                         int rblk, const float *__restrict__ x2, float *__restrict__ y1) {
+  using S = Mv3<BITS>;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
-  constexpr uint32_t MAGIC = 0x4B000000u;     // bits of 2^23
-  __shared__ float part[MV_WARPS][MV_ROWS];
+  constexpr uint32_t MAGIC = 0x4B000000u;        // bits of 2^23
+  __shared__ float part[MV3_THREADS / 32][MV3_RB];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r0 = blockIdx.x * MV_ROWS;
-  const int nr = min(MV_ROWS, d_out - r0);
+  const int nwarp = MV3_THREADS / 32, cs_n = nwarp / rblk;
+  const int rb = warp % rblk, cs = warp / rblk;
+  const int row0 = (blockIdx.x * rblk + rb) * MV3_RB;
   const int64_t words_row = static_cast<int64_t>(BITS) * d_in / 32;
   const int ng = d_in / group;
   const unsigned long long neg2 = pack2(-8388608.0f, -8388608.0f);
-  float acc[MV_ROWS];
+  // one packed step: codes at bits sh0 of h0 and sh1 of h1 against the x pair
+  auto step = [&](unsigned long long &acc2, uint32_t h0, int sh0, uint32_t h1, int sh1,
+                  unsigned long long xp) {
+    const uint32_t lo = (h0 & (MASK << sh0)) | MAGIC;
+    const uint32_t hi = (h1 & (MASK << sh1)) | MAGIC;
+    acc2 = fma2(add2(pack2(__uint_as_float(lo), __uint_as_float(hi)), neg2), xp, acc2);
+  };
+  float acc[MV3_RB];
 #pragma unroll
-  for (int k = 0; k < MV_ROWS; ++k) acc[k] = 0.f;
-  const int nchunks = (d_in + S::CHUNK - 1) / S::CHUNK;
-  for (int ch = warp; ch < nchunks; ch += MV_WARPS) {
-    const int col = ch * S::CHUNK + S::COLS * lane;
-    if (col >= d_in) continue;
-    // x pre-scaled by 2^(-BITS * position in its half word), as pairs
-    unsigned long long xp[S::COLS / 2];
+  for (int k = 0; k < MV3_RB; ++k) acc[k] = 0.f;
+  const int ntiles = (d_in + S::TILE - 1) / S::TILE;
+  for (int t = cs; t < ntiles; t += cs_n) {
+    const int c = t * S::TILE + lane * S::LCOLS;
+    if (c >= d_in) continue;
+    uint32_t w[MV3_RB][S::WORDS];
+#pragma unroll
+    for (int k = 0; k < MV3_RB; ++k) {
+      const int row = min(row0 + k, d_out - 1);
+      const uint32_t *p = codes + row * words_row + static_cast<int64_t>(c) * BITS / 32;
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
+      w[k][0] = v.x;
+      w[k][1] = v.y;
+      w[k][2] = v.z;
+      w[k][3] = v.w;
+    }
+    unsigned long long a2[MV3_RB];
+#pragma unroll
+    for (int k = 0; k < MV3_RB; ++k) a2[k] = 0ull;
     float xsum = 0.f;
-    const float4 *x4 = reinterpret_cast<const float4 *>(x2 + col);
+    {
+      constexpr int PER16 = 16 / BITS;           // codes per 16-bit half word
 #pragma unroll
+      for (int hwi = 0; hwi < 8; ++hwi) {        // half words of the 4 code words
+        const int j0 = hwi * PER16;
+        float xv[PER16];
 #pragma unroll
-    for (int q = 0; q < S::COLS / 4; ++q) {
-      const float4 v = __ldg(x4 + q);
-      xsum += (v.x + v.y) + (v.z + v.w);
-      const float e[4] = {v.x, v.y, v.z, v.w};
+        for (int q = 0; q < PER16 / 4; ++q) {
+          const float4 v = __ldg(reinterpret_cast<const float4 *>(x2 + c + j0) + q);
+          xv[4 * q] = v.x;
+          xv[4 * q + 1] = v.y;
+          xv[4 * q + 2] = v.z;
+          xv[4 * q + 3] = v.w;
+        }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j0 = 4 * q + 2 * h, j1 = j0 + 1;
-        // times 2^(-BITS * position): exact (a power of two)
-        xp[j0 / 2] = pack2(e[2 * h] * __int_as_float((127 - BITS * (j0 % PER16)) << 23),
-                           e[2 * h + 1] * __int_as_float((127 - BITS * (j1 % PER16)) << 23));
-      }
-    }
-    const int g = col / group;
-    const int64_t w0 = static_cast<int64_t>(col) * BITS / 32;
-    uint32_t w[MV_ROWS][S::WORDS];
+        for (int i = 0; i < PER16; i += 2) {
+          xsum += xv[i] + xv[i + 1];
+          const unsigned long long xp =
+              pack2(xv[i] * pow2_neg(BITS * i), xv[i + 1] * pow2_neg(BITS * (i + 1)));
 #pragma unroll
-    for (int k = 0; k < MV_ROWS; ++k) {
-      const int64_t row = r0 + kq_min(k, nr - 1);
-      const uint32_t *p = codes + row * words_row + w0;
-#pragma unroll
-      for (int t = 0; t < S::WORDS; ++t) w[k][t] = __ldg(p + t);
-    }
-#pragma unroll
-    for (int k = 0; k < MV_ROWS; ++k) {
-      const int64_t row = r0 + kq_min(k, nr - 1);
-      const float sc = __ldg(scales + row * ng + g);
-      const float z = static_cast<float>(__ldg(zeros + row * ng + g));
-      unsigned long long a2 = 0ull;
-#pragma unroll
-      for (int t = 0; t < S::WORDS; ++t) {
-#pragma unroll
-        for (int hw = 0; hw < 2; ++hw) {
-          const uint32_t h16 = hw ? (w[k][t] >> 16) : w[k][t];
-#pragma unroll
-          for (int i = 0; i < PER16; i += 2) {
-            const uint32_t lo = (h16 & (MASK << (BITS * i))) | MAGIC;
-            const uint32_t hi = (h16 & (MASK << (BITS * (i + 1)))) | MAGIC;
-            const int j = (t * 2 + hw) * PER16 + i;   // column within the lane's 16
-            a2 = fma2(add2(pack2(__uint_as_float(lo), __uint_as_float(hi)), neg2), xp[j / 2], a2);
+          for (int k = 0; k < MV3_RB; ++k) {
+            const uint32_t h = (hwi & 1) ? (w[k][hwi >> 1] >> 16) : w[k][hwi >> 1];
+            step(a2[k], h, BITS * i, h, BITS * (i + 1), xp);
           }
         }
       }
-      const float dot = __uint_as_float(static_cast<uint32_t>(a2)) +
-                        __uint_as_float(static_cast<uint32_t>(a2 >> 32));
+    }
+    const int g = c / group;
+#pragma unroll
+    for (int k = 0; k < MV3_RB; ++k) {
+      const int row = min(row0 + k, d_out - 1);
+      const float sc = __ldg(scales + static_cast<int64_t>(row) * ng + g);
+      const float z = static_cast<float>(__ldg(zeros + static_cast<int64_t>(row) * ng + g));
+      const float dot = lo_of(a2[k]) + hi_of(a2[k]);
       acc[k] = fmaf(sc, dot - z * xsum, acc[k]);
     }
   }
 #pragma unroll
-  for (int k = 0; k < MV_ROWS; ++k) {
+  for (int k = 0; k < MV3_RB; ++k) {
     const float v = warp_sum(acc[k]);
     if (lane == 0) part[warp][k] = v;
   }
   __syncthreads();
-  if (threadIdx.x < nr) {
-    float v = 0.f;
-#pragma unroll
-    for (int w2 = 0; w2 < MV_WARPS; ++w2) v += part[w2][threadIdx.x];
-    y1[r0 + threadIdx.x] = v;
+  if (threadIdx.x < rblk * MV3_RB) {
+    const int rbi = threadIdx.x / MV3_RB, k = threadIdx.x % MV3_RB;
+    const int row = (blockIdx.x * rblk + rbi) * MV3_RB + k;
+    if (row < d_out) {
+      float v = 0.f;
+      for (int c2 = 0; c2 < cs_n; ++c2) v += part[c2 * rblk + rbi][k];
+      y1[row] = v;
+    }
   }
 }
 
@@ -269,14 +302,24 @@ template <int BITS>
 kronq_status launch_gemv(cudaStream_t st, const uint32_t *codes, const float *scales,
                          const uint8_t *zeros, int64_t d_out, int64_t d_in, int group,
                          const float *x2, float *y1) {
-  const int64_t grid = ceil_div(d_out, MV_ROWS);
-  if constexpr (BITS == 3) {
-    dequant_gemv_kernel<BITS><<<static_cast<unsigned>(grid), MV_THREADS, 0, st>>>(
-        codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, x2, y1);
-  } else {
-    dequant_gemv_x2_kernel<BITS><<<static_cast<unsigned>(grid), MV_THREADS, 0, st>>>(
-        codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, x2, y1);
+  if constexpr (BITS != 3) {
+    constexpr int64_t LCOLS = Mv3<BITS>::LCOLS;
+    if (d_in % LCOLS == 0 && group % LCOLS == 0) {
+      // row blocks per CTA (the other warps split the columns): the largest
+      // that still gives every SM two CTAs
+      int rblk = 4;
+      while (rblk > 1 && ceil_div(d_out, int64_t(rblk) * MV3_RB) < 2 * 148) rblk /= 2;
+      const int64_t grid3 = ceil_div(d_out, int64_t(rblk) * MV3_RB);
+      dequant_gemv3_kernel<BITS><<<static_cast<unsigned>(grid3), MV3_THREADS, 0, st>>>(
+          codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, rblk,
+          x2, y1);
+      KQ_CHECK_LAUNCH();
+      return KRONQ_OK;
+    }
   }
+  const int64_t grid = ceil_div(d_out, MV_ROWS);
+  dequant_gemv_kernel<BITS><<<static_cast<unsigned>(grid), MV_THREADS, 0, st>>>(
+      codes, scales, zeros, static_cast<int>(d_out), static_cast<int>(d_in), group, x2, y1);
   KQ_CHECK_LAUNCH();
   return KRONQ_OK;
 }
