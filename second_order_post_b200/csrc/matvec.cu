@@ -128,15 +128,10 @@ __device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
   return d;
 }
-__device__ __forceinline__ float lo_of(unsigned long long v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float hi_of(unsigned long long v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
+__device__ __forceinline__ float2 unpack2(unsigned long long v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
 }
 __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
                                                    unsigned long long c) {
@@ -251,7 +246,8 @@ __global__ void __launch_bounds__(MV3_THREADS, 2)
       const int row = min(row0 + k, d_out - 1);
       const float sc = __ldg(scales + static_cast<int64_t>(row) * ng + g);
       const float z = static_cast<float>(__ldg(zeros + static_cast<int64_t>(row) * ng + g));
-      const float dot = lo_of(a2[k]) + hi_of(a2[k]);
+      const float2 d2 = unpack2(a2[k]);
+      const float dot = d2.x + d2.y;
       acc[k] = fmaf(sc, dot - z * xsum, acc[k]);
     }
   }
