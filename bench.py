@@ -308,7 +308,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -418,7 +418,9 @@ def main():
         Wh = W.cpu().pin_memory()
         Xh = X.cpu().pin_memory()
         Gh = G.cpu().pin_memory()
-        Wd, Xd, Gd = torch.empty_like(W), torch.empty_like(X), torch.empty_like(G)
+        # two device copies of the inputs: step i+1's copies run under step i
+        bufs = [(torch.empty_like(W), torch.empty_like(X), torch.empty_like(G))
+                for _ in range(2)]
         codes_h = torch.empty(eng.codes.shape, dtype=eng.codes.dtype, pin_memory=True)
         scales_h = torch.empty(eng.scales.shape, dtype=eng.scales.dtype, pin_memory=True)
         zeros_h = torch.empty(eng.zeros.shape, dtype=eng.zeros.dtype, pin_memory=True)
@@ -431,26 +433,30 @@ def main():
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         side.wait_event(e0)
-        freed = {}   # step name -> event after the step that last reads an input
-        for _ in range(args.e2e_steps):
-            # the inputs cross on a copy stream, X first; each copy waits only
-            # until the previous step has finished reading that buffer, so the
-            # next X lands while this sublayer's BiIP, Cholesky and OBS run
+        # per buffer set: step name -> event after the step that last read it
+        freed = [{}, {}]
+        for i in range(args.e2e_steps):
+            # the inputs cross on a copy stream, X first, into the buffer set
+            # the step before last used; each copy waits only until that
+            # step has finished reading the buffer, so the copies of the next
+            # sublayer run while this one computes
+            Wd, Xd, Gd = bufs[i % 2]
+            fr = freed[i % 2]
             arrived = {}
             with torch.cuda.stream(side):
                 for key, dst, src in (("cov_x", Xd, Xh), ("cov_g", Gd, Gh), ("biip", Wd, Wh)):
-                    if key in freed:
-                        side.wait_event(freed[key])
+                    if key in fr:
+                        side.wait_event(fr[key])
                     dst.copy_(src, non_blocking=True)
                     ev = torch.cuda.Event()
                     ev.record(side)
                     arrived[key] = ev
 
-            def mark(name):
+            def mark(name, fr=fr):
                 if name in ("cov_x", "cov_g", "biip"):
                     ev = torch.cuda.Event()
                     ev.record(stream)
-                    freed[name] = ev
+                    fr[name] = ev
 
             eng.run(Wd, Xd, Gd, mark=mark, deps=arrived)
             codes_h.copy_(eng.codes, non_blocking=True)
@@ -467,7 +473,7 @@ def main():
         e2e = {"value": world * flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": ems, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
-        del Wh, Xh, Gh, Wd, Xd, Gd
+        del Wh, Xh, Gh, Wd, Xd, Gd, bufs
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
