@@ -7,16 +7,22 @@
 //
 // Every rotation of an R x C row-major matrix M -> P_r diag(cr) M diag(cc) P_cᵀ
 // is split into memory passes whose working sets fit in shared memory:
-//   row pass      one row chunk of Lc*m_c contiguous columns per CTA: input
-//                 factors, Hadamard over the chunk's a-index, Q_m over each
-//                 group of m_c contiguous values (the whole column side when
-//                 the row fits in 112 KB)
-//   row-side Q_m  groups of m_r consecutive rows, one thread per column
-//   strided pass  Hadamard over index bits whose elements sit at a fixed
-//                 stride (within a row, or across rows); one [A][cw] slab per
-//                 CTA with cw contiguous columns
+//   row pass      one row chunk of Lc*m_c contiguous columns per CTA (or per
+//                 step of a persistent CTA): input factors, Hadamard over the
+//                 chunk's a-index, Q_m over each group of m_c contiguous
+//                 values (the whole column side when the row fits)
+//   column pass   the whole row side in one read and one write: a cluster
+//                 of CTAs holds a strip of columns over all rows, Q_m over
+//                 each group of rows, the local Hadamard, then the top bits
+//                 across the cluster through distributed shared memory
+//   row-side Q_m  groups of m_r consecutive rows (m_r > 32, when the column
+//   + strided     pass does not apply), then the Hadamard over index bits
+//                 whose elements sit at a fixed stride
 // The Hadamard factors commute with each other and with Q_m (Kronecker
-// structure), so the order of the passes does not change the result.
+// structure), and P_r and P_c act on different sides, so the order of the
+// passes does not change the result: in place on fp32 with Q_28 on the row
+// side (H_X of the pages' 70B shapes) the column pass goes first and takes
+// both diagonal factors.
 #include <math.h>
 
 #include "kernels.cuh"
@@ -939,7 +945,7 @@ kronq_status launch_colpass(cudaStream_t st, float *M, int64_t ld, int64_t R,
     K = 8;
     W4 = 2;
   }
-  // factors ride on the Q_28 MMA mix of whole 16-column strips only
+  // factors ride on the Q_28 MMA mix of whole strips only
   if ((fr || fc) && !(m == 28 && (W4 == 4 || W4 == 2) && C % (4 * W4) == 0))
     return KRONQ_ERR_UNSUPPORTED;
   const int64_t strips = ceil_div(C, 4 * W4);
