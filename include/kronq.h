@@ -195,7 +195,9 @@ kronq_status kronq_sensitivity(kronq_stream_t stream, const float *H_X,
  * s_x[d_in], s_g[d_out]: fp32 outputs, the diagonal scales used (all 1 with
  * KRONQ_FLAG_NO_SCALE). ws: kronq_workspace_bytes(KRONQ_WS_BIIP, ...).
  * Requires d_in % 32 == 0, had*m == d per side, had a power of two,
- * 1 <= m <= 256, d <= 65536. info: NONFINITE when a diagonal is not finite.
+ * 1 <= m <= 256, d <= 65536. info: NONFINITE when a diagonal is not finite;
+ * TIMEOUT when a bounded wait of a pass (a bulk copy landing) ran out (the
+ * outputs are then incomplete and must not be used).
  */
 kronq_status kronq_biip(kronq_stream_t stream, const kronq_opts *opts,
                         const void *W, kronq_dtype wdtype, int64_t d_out,
