@@ -158,7 +158,9 @@ def main():
         raise SystemExit(f"status word(s) {info}")
     print(f"{args.step} ok")
     if args.time and args.timer.ms:
-        print(json.dumps({"step": args.step, "workload": args.workload, "d": args.d,
+        shape = ({"workload": args.workload} if args.step in ("biip", "matvec")
+                 else {"d": args.d, **({"n": args.n} if args.step == "cov" else {})})
+        print(json.dumps({"step": args.step, **shape,
                           "ms_median": statistics.median(args.timer.ms),
                           "timed_calls": len(args.timer.ms)}))
 
